@@ -1,0 +1,11 @@
+"""CPU fp64 oracle: test infrastructure only (see coda_oracle.py)."""
+
+from .coda_oracle import (  # noqa: F401
+    gemm,
+    grg_backward,
+    grg_forward,
+    partial_sumsq,
+    silu,
+    swiglu_backward,
+    swiglu_forward,
+)

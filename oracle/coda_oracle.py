@@ -1,0 +1,207 @@
+"""CPU oracle for the CODA GEMM-Residual-RMSNorm-GEMM block and the SwiGLU MLP.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this
+module.  The product path (the CUDA library and its Python binding) never calls
+it and shares no code with it.
+
+Everything here is the plain, unfused definition of what the fused kernels must
+reach, evaluated in float64 with numpy on the bf16-rounded inputs (the caller
+converts bf16 tensors to float64 arrays; that conversion is exact).  Matrix
+products use ``numpy.matmul`` (BLAS) as a library primitive; nothing is blocked,
+fused or reordered beyond the textbook order of operations.
+
+Sources (the pages give no formulas; see each function for the reading taken):
+
+* toolin.ai, "CODA：LLMと初心者が光速のGPUカーネルを書けるようにする",
+  section 核心の洞察 (core insight): a GEMM-RMSNorm-GEMM block, whose RMSNorm
+  row scale r commutes with the following GEMM.
+* kucoin.com (ru), "CODA: новое исследование ...", section
+  «В «Финале» спрятаны сокровища»: the block is GEMM -> residual add -> RMS
+  normalisation -> GEMM; the first GEMM's epilogue emits per-tile partial
+  mean squares which a light reduction combines.
+* same pages, the five-primitive table (toolin.ai §組み合わせ可能な5種類の「積み木」;
+  kucoin (ru) §Пять «кирпичиков»): residual add and activation (SwiGLU) are
+  elementwise epilogue transforms.
+* toolin.ai §実験結果 and kucoin (ru) §Результаты эксперимента: the backward of
+  GEMM-Residual-PartialRMS-GEMM and of SwiGLU are the measured kernels.
+
+Readings taken where the pages are silent (all listed in the design doc):
+eps sits inside the root, r_i = 1/sqrt(mean_j H_ij^2 + eps), the mean runs over
+the full hidden width d; the first F rows of the gate/up weight are the gate
+(silu input) and the last F the up projection; weights use the [out, in]
+layout, so the pages' "X*W1" is ``X @ W1.T``; the scalar loss whose gradient the
+backward returns is <dY, Y> + <dH_in, H>.
+
+Parity pins: every function here is pinned by tests in
+``tests/test_oracle_pins.py`` (closed forms, a hand-derived worked example in
+``tests/golden/``, central finite differences, and torch fp64 library routines).
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "silu",
+    "grg_forward",
+    "grg_backward",
+    "partial_sumsq",
+    "swiglu_forward",
+    "swiglu_backward",
+    "gemm",
+]
+
+
+def _f64(x) -> np.ndarray:
+    return np.asarray(x, dtype=np.float64)
+
+
+def _sigmoid(x: np.ndarray) -> np.ndarray:
+    # Two-branch logistic so that neither branch overflows.
+    out = np.empty_like(x)
+    pos = x >= 0
+    out[pos] = 1.0 / (1.0 + np.exp(-x[pos]))
+    ex = np.exp(x[~pos])
+    out[~pos] = ex / (1.0 + ex)
+    return out
+
+
+def silu(x) -> np.ndarray:
+    """silu(x) = x * sigmoid(x), the gate nonlinearity of SwiGLU."""
+    x = _f64(x)
+    return x * _sigmoid(x)
+
+
+def gemm(A, B) -> np.ndarray:
+    """C = A @ B.T in float64 (weights in [out, in] layout)."""
+    return _f64(A) @ _f64(B).T
+
+
+def partial_sumsq(H, tile_width: int) -> np.ndarray:
+    """Per-tile partial sums of squares of H.
+
+    P[i, t] = sum over j in [t*w, (t+1)*w) of H[i, j]**2, with w = tile_width
+    and the last tile ragged when d is not a multiple of w.  This is the
+    "partial RMS" that the first GEMM's epilogue emits (kucoin (ru)
+    §«В «Финале» спрятаны сокровища»; toolin.ai five-primitive table, row
+    "tile-wise reduction: local mean square").
+    """
+    H = _f64(H)
+    M, d = H.shape
+    T = -(-d // tile_width)
+    P = np.zeros((M, T), dtype=np.float64)
+    for t in range(T):
+        blk = H[:, t * tile_width:(t + 1) * tile_width]
+        P[:, t] = np.sum(blk * blk, axis=1)
+    return P
+
+
+def grg_forward(X, W1, R, g, W2, eps: float) -> dict:
+    """GEMM -> residual -> RMSNorm(gain g) -> GEMM -> SwiGLU, unfused.
+
+    Shapes: X [M, K], W1 [d, K], R [M, d], g [d], W2 [2F, d].
+    Steps in textbook order (toolin.ai §核心の洞察; kucoin (ru)
+    §«В «Финале» спрятаны сокровища»):
+      H  = X W1^T + R                      (GEMM1 + residual add)
+      ms = mean_j H_ij^2 ;  r = 1/sqrt(ms + eps)
+      n  = diag(r) H ;  u = n * g          (RMSNorm with gain)
+      A  = u W2^T ;  a = A[:, :F], b = A[:, F:]
+      Y  = silu(a) * b                     (SwiGLU)
+    Returns every intermediate so that tests can compare each saved tensor.
+    """
+    X, W1, R, g, W2 = map(_f64, (X, W1, R, g, W2))
+    H = X @ W1.T + R
+    d = H.shape[1]
+    ms = np.sum(H * H, axis=1) / d
+    r = 1.0 / np.sqrt(ms + eps)
+    n = H * r[:, None]
+    u = n * g[None, :]
+    A = u @ W2.T
+    F = W2.shape[0] // 2
+    a = A[:, :F]
+    b = A[:, F:]
+    Y = silu(a) * b
+    return {"H": H, "ms": ms, "r": r, "n": n, "u": u, "A": A, "a": a, "b": b, "Y": Y}
+
+
+def _swiglu_grads(dY, a, b):
+    """d(silu(a)*b)/da and /db contracted with dY (chain rule, by hand)."""
+    s = _sigmoid(a)
+    dsilu = s * (1.0 + a * (1.0 - s))  # derivative of a*sigmoid(a)
+    da = dY * b * dsilu
+    db = dY * a * s
+    return da, db
+
+
+def grg_backward(dY, X, W1, R, g, W2, eps: float, dH_in=None, fwd: dict | None = None) -> dict:
+    """Gradients of L = <dY, Y> + <dH_in, H> for the block of grg_forward.
+
+    Textbook reverse-mode, one step at a time (no fused identities):
+      da, db from SwiGLU;  dA = [da | db]
+      dW2 = dA^T u ;  du = dA W2 ;  dg_j = sum_i du_ij n_ij ;  dn = du * g
+      RMSNorm:  n_ij = H_ij r_i with r_i = (ms_i + eps)^(-1/2), ms_i = mean_j H_ij^2
+                dH = r * dn - (r^3 / d) * (sum_k dn_ik H_ik) * H   (+ dH_in)
+      dR = dH ;  dX = dH W1 ;  dW1 = dH^T X
+    The pages name this backward (toolin.ai §実験結果: GEMM-Residual-PartialRMS-GEMM
+    backward; kucoin (ru) §Результаты эксперимента) but print no formula; the
+    chain rule above is the plain definition.
+    """
+    if fwd is None:
+        fwd = grg_forward(X, W1, R, g, W2, eps)
+    dY, X, W1, g, W2 = map(_f64, (dY, X, W1, g, W2))
+    H, r, n, u, a, b = fwd["H"], fwd["r"], fwd["n"], fwd["u"], fwd["a"], fwd["b"]
+    d = H.shape[1]
+    da, db = _swiglu_grads(dY, a, b)
+    dA = np.concatenate([da, db], axis=1)
+    dW2 = dA.T @ u
+    du = dA @ W2
+    dg = np.sum(du * n, axis=0)
+    dn = du * g[None, :]
+    dr = np.sum(dn * H, axis=1)               # dL/dr_i
+    dms = dr * (-0.5) * r ** 3                # dr/dms = -1/2 (ms+eps)^(-3/2)
+    dH = dn * r[:, None] + (dms[:, None] * (2.0 / d)) * H
+    if dH_in is not None:
+        dH = dH + _f64(dH_in)
+    dX = dH @ W1
+    dW1 = dH.T @ X
+    return {"dA": dA, "da": da, "db": db, "du": du, "dn": dn, "dH": dH, "dR": dH,
+            "dX": dX, "dW1": dW1, "dW2": dW2, "dg": dg}
+
+
+def swiglu_forward(X, Wgu, Wdown) -> dict:
+    """SwiGLU MLP: A = X Wgu^T, Y = silu(a) * b, Out = Y Wdown^T.
+
+    Shapes: X [M, d], Wgu [2F, d] (gate rows first), Wdown [d, F].
+    SwiGLU as an elementwise epilogue transform (toolin.ai five-primitive
+    table, "activation"; kucoin (ru) §«В «Финале» спрятаны сокровища", SwiGLU
+    named among the reparameterised operations).
+    """
+    X, Wgu, Wdown = map(_f64, (X, Wgu, Wdown))
+    A = X @ Wgu.T
+    F = Wgu.shape[0] // 2
+    a = A[:, :F]
+    b = A[:, F:]
+    Y = silu(a) * b
+    Out = Y @ Wdown.T
+    return {"A": A, "a": a, "b": b, "Y": Y, "Out": Out}
+
+
+def swiglu_backward(dOut, X, Wgu, Wdown, fwd: dict | None = None) -> dict:
+    """Gradients of L = <dOut, Out> for swiglu_forward (chain rule by hand).
+
+      dY = dOut Wdown ;  dWdown = dOut^T Y
+      da, db from SwiGLU ;  dA = [da | db]
+      dWgu = dA^T X ;  dX = dA Wgu
+    SwiGLU backward is one of the measured kernels (toolin.ai §実験結果).
+    """
+    if fwd is None:
+        fwd = swiglu_forward(X, Wgu, Wdown)
+    dOut, X, Wgu, Wdown = map(_f64, (dOut, X, Wgu, Wdown))
+    dY = dOut @ Wdown
+    dWdown = dOut.T @ fwd["Y"]
+    da, db = _swiglu_grads(dY, fwd["a"], fwd["b"])
+    dA = np.concatenate([da, db], axis=1)
+    dWgu = dA.T @ X
+    dX = dA @ Wgu
+    return {"dY": dY, "dA": dA, "da": da, "db": db, "dWgu": dWgu, "dWdown": dWdown, "dX": dX}

@@ -1,0 +1,304 @@
+"""Pins for the CPU oracle, independent of the oracle's own code (CPU only).
+
+Each test checks the oracle against something other than itself: a
+hand-derived worked example (tests/golden), closed forms, invariants of
+RMSNorm and SwiGLU, central finite differences of the scalar loss, torch fp64
+library routines (rms_norm, linear, silu, autograd), and brute-force loops on
+tiny inputs.  A plausible slip in the oracle (eps outside the root, the mean
+over a tile instead of d, gate/up swapped, a dropped RMSNorm backward term, a
+transposed weight gradient) fails at least one of them.
+"""
+
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as Fn
+
+from oracle import coda_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _ev(expr, **env):
+    return eval(expr, {"exp": math.exp, "sqrt": math.sqrt, "__builtins__": {}}, env)
+
+
+# ----------------------------------------------------------------------------- worked example
+
+def _hand():
+    with open(os.path.join(GOLDEN, "grg_hand_example.json")) as f:
+        return json.load(f)
+
+
+def test_hand_example_forward():
+    ex = _hand()
+    inp = {k: np.array(v, dtype=np.float64) for k, v in ex["inputs"].items()}
+    for key, eps in (("eps0", 0.0), ("eps1", 1.0)):
+        f = O.grg_forward(inp["X"], inp["W1"], inp["R"], inp["g"], inp["W2"], eps)
+        exp = ex["expected"][key]
+        assert f["r"][0] == pytest.approx(_ev(exp["r"]), rel=1e-15)
+        assert f["a"][0, 0] == pytest.approx(_ev(exp["a"]), rel=1e-15)
+        assert f["b"][0, 0] == pytest.approx(_ev(exp["b"]), rel=1e-15)
+        assert f["Y"][0, 0] == pytest.approx(_ev(exp["Y"]), rel=1e-14)
+        if "H" in exp:
+            np.testing.assert_array_equal(f["H"][0], [_ev(e) for e in exp["H"]])
+
+
+def test_hand_example_backward():
+    ex = _hand()
+    inp = {k: np.array(v, dtype=np.float64) for k, v in ex["inputs"].items()}
+    e = ex["expected"]["bwd_eps0"]
+    s = _ev(e["s"])
+    da = _ev(e["da"], s=s)
+    db = _ev(e["db"], s=s)
+    env = {"da": da, "db": db}
+    b = O.grg_backward(inp["dY"], inp["X"], inp["W1"], inp["R"], inp["g"], inp["W2"], 0.0)
+    np.testing.assert_allclose(b["dA"][0], [da, db], rtol=1e-14)
+    np.testing.assert_allclose(b["dH"][0], [_ev(x, **env) for x in e["dH"]], rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(b["dX"][0], [_ev(x, **env) for x in e["dH"]], rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(b["dW1"], [[_ev(x, **env) for x in row] for row in e["dW1"]], rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(b["dW2"], [[_ev(x, **env) for x in row] for row in e["dW2"]], rtol=1e-14)
+    np.testing.assert_allclose(b["dg"], [_ev(x, **env) for x in e["dg"]], rtol=1e-14)
+
+
+# ----------------------------------------------------------------------------- closed forms
+
+def test_constant_rows_closed_form_r():
+    """X = 0 and R_i = c_i * ones  =>  H_i = c_i, r_i = 1/sqrt(c_i^2 + eps).
+
+    Distinguishes eps inside vs outside the root and mean over d vs a sum.
+    """
+    M, K, d, F = 5, 8, 12, 3
+    c = np.array([0.5, -1.0, 2.0, 3.0, 1e-3])
+    R = c[:, None] * np.ones((1, d))
+    X = np.zeros((M, K))
+    rng = np.random.default_rng(1)
+    W1 = rng.standard_normal((d, K))
+    W2 = rng.standard_normal((2 * F, d))
+    g = 1 + 0.1 * rng.standard_normal(d)
+    for eps in (1e-6, 0.25):
+        f = O.grg_forward(X, W1, R, g, W2, eps)
+        np.testing.assert_allclose(f["r"], 1.0 / np.sqrt(c * c + eps), rtol=1e-14)
+
+
+def test_unit_rms_rows_when_gain_is_one():
+    """g = 1: mean_j n_ij^2 = ms_i / (ms_i + eps); exactly 1 at eps = 0."""
+    rng = np.random.default_rng(2)
+    M, K, d, F = 7, 16, 24, 5
+    X, R = rng.standard_normal((M, K)), rng.standard_normal((M, d))
+    W1, W2 = rng.standard_normal((d, K)), rng.standard_normal((2 * F, d))
+    g = np.ones(d)
+    f0 = O.grg_forward(X, W1, R, g, W2, 0.0)
+    np.testing.assert_allclose(np.mean(f0["n"] ** 2, axis=1), 1.0, rtol=1e-13)
+    eps = 0.3
+    f1 = O.grg_forward(X, W1, R, g, W2, eps)
+    ms = np.mean(f1["H"] ** 2, axis=1)
+    np.testing.assert_allclose(np.mean(f1["n"] ** 2, axis=1), ms / (ms + eps), rtol=1e-13)
+
+
+def test_scale_invariance_at_zero_eps():
+    """RMSNorm(alpha H) = RMSNorm(H) when eps = 0, so Y is unchanged by scaling X and R."""
+    rng = np.random.default_rng(3)
+    M, K, d, F = 4, 8, 8, 6
+    X, R = rng.standard_normal((M, K)), rng.standard_normal((M, d))
+    W1, W2 = rng.standard_normal((d, K)), rng.standard_normal((2 * F, d))
+    g = 1 + 0.1 * rng.standard_normal(d)
+    y1 = O.grg_forward(X, W1, R, g, W2, 0.0)["Y"]
+    y2 = O.grg_forward(3.5 * X, W1, 3.5 * R, g, W2, 0.0)["Y"]
+    np.testing.assert_allclose(y1, y2, rtol=1e-12, atol=1e-14)
+
+
+def test_row_scale_commutes_with_second_gemm():
+    """The CODA identity: diag(r) (H (diag(g) W2^T)) equals RMSNorm(H)*g times W2^T.
+
+    The oracle computes the right-hand side in textbook order; the test
+    evaluates the left-hand side (r deferred past the GEMM, g folded into W2).
+    """
+    rng = np.random.default_rng(4)
+    M, K, d, F = 9, 12, 16, 10
+    X, R = rng.standard_normal((M, K)), rng.standard_normal((M, d))
+    W1, W2 = rng.standard_normal((d, K)), rng.standard_normal((2 * F, d))
+    g = 1 + 0.1 * rng.standard_normal(d)
+    f = O.grg_forward(X, W1, R, g, W2, 1e-5)
+    W2g = W2 * g[None, :]
+    lhs = f["r"][:, None] * (f["H"] @ W2g.T)
+    np.testing.assert_allclose(lhs, f["A"], rtol=1e-12, atol=1e-12)
+
+
+def test_gate_up_order_closed_form():
+    """F = d, W2 = [I; 2I], g = 1: a = n, b = 2n, Y = silu(n) * 2n (gate = first F rows)."""
+    rng = np.random.default_rng(5)
+    M, K, d = 6, 8, 8
+    X, R = rng.standard_normal((M, K)), rng.standard_normal((M, d))
+    W1 = rng.standard_normal((d, K))
+    W2 = np.concatenate([np.eye(d), 2 * np.eye(d)], axis=0)
+    f = O.grg_forward(X, W1, R, np.ones(d), W2, 1e-6)
+    n = f["n"]
+    np.testing.assert_allclose(f["Y"], n / (1 + np.exp(-n)) * 2 * n, rtol=1e-13, atol=1e-15)
+
+
+def test_silu_special_values():
+    assert O.silu(0.0) == 0.0
+    assert O.silu(1.0) == pytest.approx(1 / (1 + math.exp(-1)), rel=1e-15)
+    x = np.linspace(-40, 40, 161)
+    np.testing.assert_allclose(O.silu(x) - O.silu(-x), x, atol=1e-13)  # silu(x) - silu(-x) = x
+    assert O.silu(-745.0) == pytest.approx(-745.0 * math.exp(-745.0), rel=1e-6, abs=1e-300)
+    assert O.silu(800.0) == 800.0
+
+
+def test_partial_sumsq_one_hot_and_totals():
+    """One-hot H puts v^2 in exactly one (row, tile) cell; tiles sum to d * ms."""
+    M, d, w = 3, 10, 4  # ragged last tile of width 2
+    for (i, j, v) in [(0, 0, 3.0), (1, 5, -2.0), (2, 9, 0.5)]:
+        H = np.zeros((M, d))
+        H[i, j] = v
+        P = O.partial_sumsq(H, w)
+        assert P.shape == (M, 3)
+        expect = np.zeros_like(P)
+        expect[i, j // w] = v * v
+        np.testing.assert_array_equal(P, expect)
+    rng = np.random.default_rng(6)
+    H = rng.standard_normal((M, d))
+    np.testing.assert_allclose(O.partial_sumsq(H, w).sum(axis=1), np.einsum("ij,ij->i", H, H), rtol=1e-14)
+
+
+def test_gemm_brute_force():
+    rng = np.random.default_rng(7)
+    A, B = rng.standard_normal((3, 5)), rng.standard_normal((4, 5))
+    C = O.gemm(A, B)
+    for i in range(3):
+        for j in range(4):
+            s = 0.0
+            for k in range(5):
+                s += A[i, k] * B[j, k]
+            assert C[i, j] == pytest.approx(s, rel=1e-13, abs=1e-14)
+
+
+# ----------------------------------------------------------------------------- finite differences
+
+def _grg_loss(p, dY, dH_in, eps):
+    f = O.grg_forward(p["X"], p["W1"], p["R"], p["g"], p["W2"], eps)
+    return float(np.sum(dY * f["Y"]) + np.sum(dH_in * f["H"]))
+
+
+def _fd_check(loss_fn, params, grads, names, h_rel=1e-6, tol=2e-6):
+    for name in names:
+        x = params[name]
+        num = np.zeros_like(x)
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            h = h_rel * max(1.0, abs(x[idx]))
+            old = x[idx]
+            x[idx] = old + h
+            lp = loss_fn(params)
+            x[idx] = old - h
+            lm = loss_fn(params)
+            x[idx] = old
+            num[idx] = (lp - lm) / (2 * h)
+        scale = max(1.0, float(np.max(np.abs(num))))
+        err = float(np.max(np.abs(num - grads[name])))
+        assert err <= tol * scale, f"d{name}: max |fd - oracle| = {err:.3e} (scale {scale:.3e})"
+
+
+def test_grg_backward_finite_differences():
+    rng = np.random.default_rng(8)
+    M, K, d, F = 3, 5, 6, 4
+    p = {
+        "X": rng.standard_normal((M, K)),
+        "W1": rng.standard_normal((d, K)) / np.sqrt(K),
+        "R": rng.standard_normal((M, d)),
+        "g": 1 + 0.1 * rng.standard_normal(d),
+        "W2": rng.standard_normal((2 * F, d)) / np.sqrt(d),
+    }
+    dY = rng.standard_normal((M, F))
+    dH_in = rng.standard_normal((M, d))
+    eps = 0.1  # large enough that a dropped eps term would show
+    b = O.grg_backward(dY, p["X"], p["W1"], p["R"], p["g"], p["W2"], eps, dH_in=dH_in)
+    grads = {"X": b["dX"], "W1": b["dW1"], "R": b["dR"], "g": b["dg"], "W2": b["dW2"]}
+    _fd_check(lambda q: _grg_loss(q, dY, dH_in, eps), p, grads, ["X", "W1", "R", "g", "W2"])
+
+
+def test_swiglu_backward_finite_differences():
+    rng = np.random.default_rng(9)
+    M, d, F = 3, 5, 4
+    p = {
+        "X": rng.standard_normal((M, d)),
+        "Wgu": rng.standard_normal((2 * F, d)) / np.sqrt(d),
+        "Wdown": rng.standard_normal((d, F)) / np.sqrt(F),
+    }
+    dOut = rng.standard_normal((M, d))
+
+    def loss(q):
+        return float(np.sum(dOut * O.swiglu_forward(q["X"], q["Wgu"], q["Wdown"])["Out"]))
+
+    b = O.swiglu_backward(dOut, p["X"], p["Wgu"], p["Wdown"])
+    grads = {"X": b["dX"], "Wgu": b["dWgu"], "Wdown": b["dWdown"]}
+    _fd_check(loss, p, grads, ["X", "Wgu", "Wdown"])
+
+
+# ----------------------------------------------------------------------------- library cross-check
+
+def test_torch_fp64_library_crosscheck_grg():
+    """torch CPU fp64: linear + rms_norm(weight=g) + linear + silu, autograd for the backward."""
+    torch.manual_seed(10)
+    M, K, d, F, eps = 16, 32, 48, 40, 1e-5
+    X = torch.randn(M, K, dtype=torch.float64, requires_grad=True)
+    W1 = (torch.randn(d, K, dtype=torch.float64) / K ** 0.5).requires_grad_()
+    R = torch.randn(M, d, dtype=torch.float64, requires_grad=True)
+    g = (1 + 0.1 * torch.randn(d, dtype=torch.float64)).requires_grad_()
+    W2 = (torch.randn(2 * F, d, dtype=torch.float64) / d ** 0.5).requires_grad_()
+    dY = torch.randn(M, F, dtype=torch.float64)
+    dH_in = torch.randn(M, d, dtype=torch.float64)
+    H = Fn.linear(X, W1) + R
+    H.retain_grad()
+    A = Fn.linear(Fn.rms_norm(H, (d,), weight=g, eps=eps), W2)
+    Y = Fn.silu(A[:, :F]) * A[:, F:]
+    ((Y * dY).sum() + (H * dH_in).sum()).backward()
+
+    npy = lambda t: t.detach().numpy()
+    f = O.grg_forward(npy(X), npy(W1), npy(R), npy(g), npy(W2), eps)
+    np.testing.assert_allclose(f["H"], npy(H), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(f["A"], npy(A), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(f["Y"], npy(Y), rtol=1e-12, atol=1e-12)
+    b = O.grg_backward(npy(dY), npy(X), npy(W1), npy(R), npy(g), npy(W2), eps, dH_in=npy(dH_in), fwd=f)
+    for mine, ref in (("dX", X), ("dW1", W1), ("dR", R), ("dg", g), ("dW2", W2)):
+        np.testing.assert_allclose(b[mine], ref.grad.numpy(), rtol=1e-10, atol=1e-11, err_msg=mine)
+
+
+def test_torch_fp64_library_crosscheck_swiglu():
+    torch.manual_seed(11)
+    M, d, F = 16, 32, 24
+    X = torch.randn(M, d, dtype=torch.float64, requires_grad=True)
+    Wgu = (torch.randn(2 * F, d, dtype=torch.float64) / d ** 0.5).requires_grad_()
+    Wdown = (torch.randn(d, F, dtype=torch.float64) / F ** 0.5).requires_grad_()
+    dOut = torch.randn(M, d, dtype=torch.float64)
+    A = Fn.linear(X, Wgu)
+    Out = Fn.linear(Fn.silu(A[:, :F]) * A[:, F:], Wdown)
+    (Out * dOut).sum().backward()
+    npy = lambda t: t.detach().numpy()
+    f = O.swiglu_forward(npy(X), npy(Wgu), npy(Wdown))
+    np.testing.assert_allclose(f["Out"], npy(Out), rtol=1e-12, atol=1e-12)
+    b = O.swiglu_backward(npy(dOut), npy(X), npy(Wgu), npy(Wdown), fwd=f)
+    for mine, ref in (("dX", X), ("dWgu", Wgu), ("dWdown", Wdown)):
+        np.testing.assert_allclose(b[mine], ref.grad.numpy(), rtol=1e-10, atol=1e-11, err_msg=mine)
+
+
+def test_row_locality_of_forward_and_row_gradients():
+    """Permuting token rows permutes H, r, Y, dX, dR and leaves the weight gradients unchanged."""
+    rng = np.random.default_rng(12)
+    M, K, d, F = 6, 8, 8, 4
+    X, R = rng.standard_normal((M, K)), rng.standard_normal((M, d))
+    W1, W2 = rng.standard_normal((d, K)), rng.standard_normal((2 * F, d))
+    g = 1 + 0.1 * rng.standard_normal(d)
+    dY = rng.standard_normal((M, F))
+    perm = rng.permutation(M)
+    b0 = O.grg_backward(dY, X, W1, R, g, W2, 1e-6)
+    b1 = O.grg_backward(dY[perm], X[perm], W1, R[perm], g, W2, 1e-6)
+    np.testing.assert_allclose(b1["dX"], b0["dX"][perm], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(b1["dW2"], b0["dW2"], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(b1["dg"], b0["dg"], rtol=1e-12, atol=1e-12)
