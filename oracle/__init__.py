@@ -2,6 +2,11 @@
 
 from .coda_oracle import (  # noqa: F401
     gemm,
+    grg_backward_stored,
+    grg_forward_stored,
+    round_bf16,
+    swiglu_backward_stored,
+    swiglu_forward_stored,
     grg_backward,
     grg_forward,
     partial_sumsq,

@@ -50,6 +50,11 @@ __all__ = [
     "swiglu_forward",
     "swiglu_backward",
     "gemm",
+    "round_bf16",
+    "grg_forward_stored",
+    "grg_backward_stored",
+    "swiglu_forward_stored",
+    "swiglu_backward_stored",
 ]
 
 
@@ -205,3 +210,108 @@ def swiglu_backward(dOut, X, Wgu, Wdown, fwd: dict | None = None) -> dict:
     dWgu = dA.T @ X
     dX = dA @ Wgu
     return {"dY": dY, "dA": dA, "da": da, "db": db, "dWgu": dWgu, "dWdown": dWdown, "dX": dX}
+
+
+# ----------------------------------------------------------------------------- storage precision
+#
+# The method keeps every tensor it hands from one pass to the next in HBM as
+# bf16: GEMM1's epilogue stores H and GEMM2 reads it back (toolin.ai
+# §核心の洞察; kucoin (ru) §«В «Финале» спрятаны сокровища»: H goes to memory, r is
+# deferred to GEMM2's epilogue), the saved activations of the matrix-tile
+# store primitive (five-primitive table) are bf16, and every GEMM consumes
+# bf16 operands.  The *_stored functions below evaluate the same definitions
+# in float64 but round each stored tensor with ``store`` (default: round to
+# nearest bf16, ties to even) at the point where the method stores it.  With
+# ``store=lambda x: x`` they reduce to the textbook functions above (pinned).
+
+
+def round_bf16(x) -> np.ndarray:
+    """Round float64 values to the nearest bfloat16 (8 significant bits), ties to even.
+
+    x = m * 2**e with 0.5 <= |m| < 1; keeping 8 significant bits means rounding
+    m * 2**8 to an integer (numpy.rint rounds halves to even).  Values stay in
+    bf16's normal range here (|x| between 1e-30 and 1e30), so no exponent
+    clamping is needed; zeros pass through.
+    """
+    x = _f64(x)
+    m, e = np.frexp(x)
+    return np.ldexp(np.rint(m * 256.0) / 256.0, e)
+
+
+def _ident(x):
+    return x
+
+
+def grg_forward_stored(X, W1, R, g, W2, eps: float, store=round_bf16) -> dict:
+    """grg_forward with the method's dataflow at storage precision.
+
+      H   = store(X W1^T + R)                  stored by GEMM1, read by the rest
+      r   = 1/sqrt(mean_j H_ij^2 + eps)        from the stored H
+      W2g = store(W2 diag(g))                  the gain folded into GEMM2's weight
+      A   = diag(r) (H W2g^T)                  r deferred past GEMM2 (the pages' identity)
+      a, b = A[:, :F], A[:, F:];  Y = silu(a) * b   (Y from the unrounded a, b)
+      a_s, b_s = store(a), store(b)            saved for the backward
+    """
+    X, W1, R, g, W2 = map(_f64, (X, W1, R, g, W2))
+    H = store(X @ W1.T + R)
+    d = H.shape[1]
+    ms = np.sum(H * H, axis=1) / d
+    r = 1.0 / np.sqrt(ms + eps)
+    W2g = store(W2 * g[None, :])
+    A = r[:, None] * (H @ W2g.T)
+    F = W2.shape[0] // 2
+    a, b = A[:, :F], A[:, F:]
+    Y = silu(a) * b
+    return {"H": H, "r": r, "A": A, "a": a, "b": b, "a_s": store(a), "b_s": store(b), "Y": Y}
+
+
+def grg_backward_stored(dY, X, W1, R, g, W2, eps: float, dH_in=None, store=round_bf16,
+                        fwd: dict | None = None) -> dict:
+    """grg_backward at storage precision: the same chain rule, fed by the stored
+    forward tensors (H, a, b), with the SwiGLU gradient stored once in units of
+    r_i ([da | db] scaled by the row's r, the operand of the two GEMMs that
+    consume it) and dH stored before the dX / dW1 GEMMs read it.
+    """
+    if fwd is None:
+        fwd = grg_forward_stored(X, W1, R, g, W2, eps, store)
+    dY, X, W1, g, W2 = map(_f64, (dY, X, W1, g, W2))
+    H, r, a, b = fwd["H"], fwd["r"], fwd["a_s"], fwd["b_s"]
+    d = H.shape[1]
+    n = H * r[:, None]
+    u = n * g[None, :]
+    da, db = _swiglu_grads(dY, a, b)
+    dA = np.concatenate([da, db], axis=1)
+    dA = store(dA * r[:, None]) / r[:, None]
+    dW2 = dA.T @ u
+    du = dA @ W2
+    dg = np.sum(du * n, axis=0)
+    dn = du * g[None, :]
+    dr = np.sum(dn * H, axis=1)
+    dH = dn * r[:, None] + (dr * (-0.5) * r ** 3)[:, None] * (2.0 / d) * H
+    if dH_in is not None:
+        dH = dH + _f64(dH_in)
+    dHs = store(dH)
+    return {"dA": dA, "dH": dH, "dR": dH, "dX": dHs @ W1, "dW1": dHs.T @ X, "dW2": dW2, "dg": dg}
+
+
+def swiglu_forward_stored(X, Wgu, Wdown, store=round_bf16) -> dict:
+    """swiglu_forward with Y stored before the down GEMM and a, b saved stored."""
+    X, Wgu, Wdown = map(_f64, (X, Wgu, Wdown))
+    A = X @ Wgu.T
+    F = Wgu.shape[0] // 2
+    a, b = A[:, :F], A[:, F:]
+    Y = silu(a) * b
+    Ys = store(Y)
+    return {"A": A, "a": a, "b": b, "a_s": store(a), "b_s": store(b), "Y": Y, "Y_s": Ys, "Out": Ys @ Wdown.T}
+
+
+def swiglu_backward_stored(dOut, X, Wgu, Wdown, store=round_bf16, fwd: dict | None = None) -> dict:
+    """swiglu_backward fed by the stored Y, a, b, with [da | db] stored before
+    the dWgu / dX GEMMs read it."""
+    if fwd is None:
+        fwd = swiglu_forward_stored(X, Wgu, Wdown, store)
+    dOut, X, Wgu, Wdown = map(_f64, (dOut, X, Wgu, Wdown))
+    dY = dOut @ Wdown
+    da, db = _swiglu_grads(dY, fwd["a_s"], fwd["b_s"])
+    dA = store(np.concatenate([da, db], axis=1))
+    return {"dY": dY, "dA": dA, "dWdown": dOut.T @ fwd["Y_s"], "dWgu": dA.T @ X, "dX": dA @ Wgu}

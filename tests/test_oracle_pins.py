@@ -302,3 +302,60 @@ def test_row_locality_of_forward_and_row_gradients():
     np.testing.assert_allclose(b1["dX"], b0["dX"][perm], rtol=1e-12, atol=1e-13)
     np.testing.assert_allclose(b1["dW2"], b0["dW2"], rtol=1e-12, atol=1e-12)
     np.testing.assert_allclose(b1["dg"], b0["dg"], rtol=1e-12, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- storage precision
+
+def test_round_bf16_matches_library_conversion_and_ties():
+    """round_bf16 equals torch's float32 -> bfloat16 conversion (round to nearest even)."""
+    gen = torch.Generator().manual_seed(13)
+    x = torch.randn(200000, generator=gen, dtype=torch.float32) * torch.exp(torch.randn(200000, generator=gen) * 4)
+    ref = x.to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(O.round_bf16(x.double().numpy()), ref)
+    # Hand ties: the bf16 spacing at 1 is 2^-7, so 1 + 2^-8 is halfway and goes to even (1.0);
+    # 1 + 3*2^-8 is halfway between 1 + 2^-7 (odd) and 1 + 2^-6 (even).
+    np.testing.assert_array_equal(O.round_bf16([1 + 2 ** -8, 1 + 3 * 2 ** -8, -(1 + 2 ** -8), 0.0, 3.0]),
+                                  [1.0, 1 + 2 ** -6, -1.0, 0.0, 3.0])
+
+
+def _ident(x):
+    return x
+
+
+def test_stored_functions_reduce_to_textbook_without_rounding():
+    rng = np.random.default_rng(14)
+    M, K, d, F, eps = 9, 16, 24, 10, 1e-5
+    X, R = rng.standard_normal((M, K)), rng.standard_normal((M, d))
+    W1, W2 = rng.standard_normal((d, K)) / 4, rng.standard_normal((2 * F, d)) / 5
+    g = 1 + 0.1 * rng.standard_normal(d)
+    dY, dH_in = rng.standard_normal((M, F)), rng.standard_normal((M, d))
+    f0 = O.grg_forward(X, W1, R, g, W2, eps)
+    f1 = O.grg_forward_stored(X, W1, R, g, W2, eps, store=_ident)
+    for k in ("H", "r", "a", "b", "Y"):
+        np.testing.assert_allclose(f1[k], f0[k], rtol=1e-12, atol=1e-12, err_msg=k)
+    b0 = O.grg_backward(dY, X, W1, R, g, W2, eps, dH_in=dH_in)
+    b1 = O.grg_backward_stored(dY, X, W1, R, g, W2, eps, dH_in=dH_in, store=_ident)
+    for k in ("dX", "dR", "dW1", "dW2", "dg"):
+        np.testing.assert_allclose(b1[k], b0[k], rtol=1e-11, atol=1e-11, err_msg=k)
+    Wgu, Wdown, dOut = rng.standard_normal((2 * F, d)) / 5, rng.standard_normal((d, F)) / 3, rng.standard_normal((M, d))
+    s0 = O.swiglu_forward(R, Wgu, Wdown)
+    s1 = O.swiglu_forward_stored(R, Wgu, Wdown, store=_ident)
+    np.testing.assert_allclose(s1["Out"], s0["Out"], rtol=1e-12, atol=1e-12)
+    t0 = O.swiglu_backward(dOut, R, Wgu, Wdown)
+    t1 = O.swiglu_backward_stored(dOut, R, Wgu, Wdown, store=_ident)
+    for k in ("dX", "dWgu", "dWdown"):
+        np.testing.assert_allclose(t1[k], t0[k], rtol=1e-12, atol=1e-12, err_msg=k)
+
+
+def test_stored_rounding_is_small_and_present():
+    """bf16 storage moves results by about the bf16 unit (2^-8), not more, not zero."""
+    rng = np.random.default_rng(15)
+    M, K, d, F, eps = 64, 64, 64, 64, 1e-6
+    X, R = rng.standard_normal((M, K)), rng.standard_normal((M, d))
+    W1, W2 = rng.standard_normal((d, K)) / 8, rng.standard_normal((2 * F, d)) / 8
+    g = 1 + 0.1 * rng.standard_normal(d)
+    f0 = O.grg_forward(X, W1, R, g, W2, eps)
+    f1 = O.grg_forward_stored(X, W1, R, g, W2, eps)
+    assert np.array_equal(f1["H"], O.round_bf16(f0["H"]))
+    rel = np.sqrt(np.mean((f1["A"] - f0["A"]) ** 2)) / np.sqrt(np.mean(f0["A"] ** 2))
+    assert 1e-4 < rel < 2 ** -8
