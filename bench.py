@@ -1,0 +1,476 @@
+#!/usr/bin/env python
+"""Throughput of the fused GEMM-Residual-RMSNorm-GEMM(+SwiGLU) block on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic
+LLaMA-shaped input: for the GRG workloads the gain fold, GEMM1 + residual +
+partial RMS, the row reduce, GEMM2 + r + SwiGLU, and (fwd+bwd workloads) the
+SwiGLU backward + row statistic, the dn GEMM, the dg column reduce, the dW2,
+dX and dW1 GEMMs.  All of it runs in libcoda.so through the C ABI.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 7B|70B|1B|swiglu|tiny]
+  python bench.py --impl reference ...   (the fp64 CPU oracle on the host cores)
+
+Prints one JSON line on rank 0.  Under torchrun each rank runs an independent
+replica on its own GPU (the block has no exchange step on one GPU's worth of
+tokens); value = all ranks' FLOPs / max-over-ranks device time.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fused GEMM-RMSNorm-GEMM fwd+bwd TFLOP/s and % of B200 bf16 tensor peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+WORKLOADS = {
+    "tiny": ("grg", dict(M=256, K=512, d=512, F=1024, eps=1e-6), True),
+    "1B": ("grg", dict(M=8192, K=2048, d=2048, F=8192, eps=1e-6), False),
+    "7B": ("grg", dict(M=8192, K=4096, d=4096, F=11008, eps=1e-6), True),
+    "70B": ("grg", dict(M=4096, K=8192, d=8192, F=28672, eps=1e-5), True),
+    "swiglu": ("swiglu", dict(M=16384, d=4096, F=14336), True),
+}
+
+
+def _args():
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=100)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["coda", "reference"], default="coda")
+    p.add_argument("--workload", choices=sorted(WORKLOADS), default="7B")
+    p.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed oracle sample")
+    p.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
+    return p.parse_args()
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def _flops(kind, s, bwd):
+    if kind == "grg":
+        fwd = 2.0 * s["M"] * s["K"] * s["d"] + 2.0 * s["M"] * s["d"] * 2 * s["F"]
+    else:
+        fwd = 2.0 * s["M"] * s["d"] * 2 * s["F"] + 2.0 * s["M"] * s["F"] * s["d"]
+    return fwd * (3.0 if bwd else 1.0)
+
+
+def _describe(name, kind, s, bwd):
+    if kind == "grg":
+        what = f"GEMM-Residual-RMSNorm-GEMM-SwiGLU {name} {'fwd+bwd' if bwd else 'fwd'}"
+    else:
+        what = "SwiGLU MLP fwd+bwd"
+    return {"workload": what, **s, "global_batch": s["M"]}
+
+
+# ----------------------------------------------------------------------------- CPU oracle timing
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def _oracle_step(kind, s, bwd, inputs, rows):
+    """The fp64 oracle over the first `rows` tokens of the workload (forward row-local,
+    weight gradients summed over those rows only)."""
+    from oracle import coda_oracle as O
+    if kind == "grg":
+        X, R, dY = inputs["X"][:rows], inputs["R"][:rows], inputs["dY"][:rows]
+        fwd = O.grg_forward(X, inputs["W1"], R, inputs["g"], inputs["W2"], s["eps"])
+        if bwd:
+            O.grg_backward(dY, X, inputs["W1"], R, inputs["g"], inputs["W2"], s["eps"], fwd=fwd)
+    else:
+        X, dOut = inputs["X"][:rows], inputs["dOut"][:rows]
+        fwd = O.swiglu_forward(X, inputs["Wgu"], inputs["Wdown"])
+        if bwd:
+            O.swiglu_backward(dOut, X, inputs["Wgu"], inputs["Wdown"], fwd=fwd)
+
+
+def _oracle_inputs(kind, s):
+    """Seeded inputs in float64 for the oracle (first rows only are used)."""
+    import torch
+    from gemm_epilogue_fusion_tmem_b200 import synth
+    if kind == "grg":
+        t = synth.grg_inputs(s["M"], s["K"], s["d"], s["F"], seed=0)
+    else:
+        t = synth.swiglu_inputs(s["M"], s["d"], s["F"], seed=0)
+    return {k: v.to(torch.float64).numpy() for k, v in t.items()}
+
+
+def cpu_baseline(kind, s, bwd, inputs=None, target_s=12.0):
+    inputs = inputs if inputs is not None else _oracle_inputs(kind, s)
+    # Probe on a few rows to size the bounded sample.
+    probe = min(64, s["M"])
+    t0 = time.perf_counter()
+    _oracle_step(kind, s, bwd, inputs, probe)
+    dt = max(time.perf_counter() - t0, 1e-3)
+    rate = _flops(kind, dict(s, M=probe), bwd) / dt
+    rows = max(probe, min(s["M"], int(target_s * rate / _flops(kind, dict(s, M=1), bwd))))
+    t0 = time.perf_counter()
+    _oracle_step(kind, s, bwd, inputs, rows)
+    dt = time.perf_counter() - t0
+    fl = _flops(kind, dict(s, M=rows), bwd)
+    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"fp64 numpy oracle, unfused textbook {'fwd+bwd' if bwd else 'fwd'} on the first {rows} "
+                      f"of {s['M']} tokens with the full weights ({fl / 1e12:.3f} TFLOP in {dt:.1f} s)"}
+
+
+# ----------------------------------------------------------------------------- clocks
+
+CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+class ClockSampler:
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={CLOCK_FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out = ""
+
+    def summary(self):
+        sm, mx, pw, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in (self.out or "").splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+                pw.append(float(f[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        # Median over the samples taken under load (power above 30% of the highest seen).
+        hot = [c for c, p in zip(sm, pw) if p >= 0.3 * max(pw)] or sm
+        return {"sm_mhz": statistics.median(hot), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm), "samples_under_load": len(hot), "power_w_max": max(pw)}
+
+
+# ----------------------------------------------------------------------------- traffic record
+
+def _kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "gemm_epilogue_fusion_tmem_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def _recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch recorded from an ncu capture, if taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    try:
+        with open(path) as f:
+            for line in f:
+                parts = line.split()
+                if len(parts) >= 4 and parts[0] == kernel and parts[1] == workload:
+                    return float(parts[2]) if parts[3] == _kernel_source_hash() else None
+    except OSError:
+        pass
+    return None
+
+
+# ----------------------------------------------------------------------------- the CUDA arm
+
+def _setup(kind, s, bwd, device):
+    import torch
+    from gemm_epilogue_fusion_tmem_b200 import synth
+    if kind == "grg":
+        host = synth.grg_inputs(s["M"], s["K"], s["d"], s["F"], seed=0)
+        if not bwd:
+            host.pop("dY")
+    else:
+        host = synth.swiglu_inputs(s["M"], s["d"], s["F"], seed=0)
+    dev = {k: v.to(device) for k, v in host.items()}
+    return host, dev
+
+
+def _make_step(kind, s, bwd, dev):
+    """Returns (step, outputs, launches_per_step, result_keys)."""
+    import torch
+    from gemm_epilogue_fusion_tmem_b200 import binding as B
+    lib = B.library()
+    M = s["M"]
+    if kind == "grg":
+        K, d, F = s["K"], s["d"], s["F"]
+        N = 2 * F
+        ws = B.Workspace(max(lib.coda_grg_fwd_workspace_bytes(M, K, d, N, 0),
+                             lib.coda_grg_bwd_workspace_bytes(M, K, d, N)), dev["X"].device)
+        fo = {"H": torch.empty(M, d, dtype=torch.bfloat16, device=dev["X"].device),
+              "r": torch.empty(M, dtype=torch.float32, device=dev["X"].device),
+              "Y": torch.empty(M, F, dtype=torch.bfloat16, device=dev["X"].device),
+              "AB": torch.empty(M, N, dtype=torch.bfloat16, device=dev["X"].device)}
+        bo = {}
+        if bwd:
+            bo = {"dX": torch.empty(M, K, dtype=torch.bfloat16, device=dev["X"].device),
+                  "dR": torch.empty(M, d, dtype=torch.bfloat16, device=dev["X"].device),
+                  "dW1": torch.empty(d, K, dtype=torch.bfloat16, device=dev["X"].device),
+                  "dW2": torch.empty(N, d, dtype=torch.bfloat16, device=dev["X"].device),
+                  "dg": torch.empty(d, dtype=torch.float32, device=dev["X"].device)}
+
+        def step():
+            B.grg_fwd(dev["X"], dev["W1"], dev["R"], dev["g"], dev["W2"], s["eps"], out=fo, ws=ws)
+            if bwd:
+                B.grg_bwd(dev["dY"], dev["X"], dev["W1"], fo["H"], fo["r"], fo["AB"], dev["g"], dev["W2"],
+                          out=bo, ws=ws)
+
+        outs = {**fo, **bo}
+        keys = ["Y", "dX", "dR", "dW1", "dW2", "dg"] if bwd else ["Y", "H", "r"]
+        return step, outs, (10 if bwd else 4), keys, ws
+    d, F = s["d"], s["F"]
+    ws = B.Workspace(lib.coda_swiglu_bwd_workspace_bytes(M, d, F), dev["X"].device)
+    fo, bo = {}, {}
+
+    def step():
+        B.swiglu_fwd(dev["X"], dev["Wgu"], dev["Wdown"], out=fo, ws=ws)
+        B.swiglu_bwd(dev["dOut"], dev["X"], dev["Wgu"], dev["Wdown"], fo["Y"], fo["AB"], out=bo, ws=ws)
+
+    step()  # allocate outputs once
+    outs = {**fo, **bo}
+    return step, outs, 6, ["Out", "dX", "dWgu", "dWdown"], ws
+
+
+def _dominant_kernel(kind, s, dev, outs, reps=20):
+    """Time the dominant kernel alone: the gate/up GEMM with the r + SwiGLU epilogue."""
+    import torch
+    from gemm_epilogue_fusion_tmem_b200 import binding as B
+    if kind == "grg":
+        A, W, r = outs["H"], dev["W2"], outs["r"]  # same shape and work as GEMM2 on W2g
+        K = s["d"]
+    else:
+        A, W, r = dev["X"], dev["Wgu"], None
+        K = s["d"]
+    M, F = s["M"], s["F"]
+    o = {"Y": torch.empty(M, F, dtype=torch.bfloat16, device=A.device),
+         "AB": torch.empty(M, 2 * F, dtype=torch.bfloat16, device=A.device)}
+    for _ in range(3):
+        B.gemm_swiglu(A, W, r, out=o)
+    st = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(st)
+    for _ in range(reps):
+        B.gemm_swiglu(A, W, r, out=o)
+    e1.record(st)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    flops = 2.0 * M * K * 2 * F
+    return "gemm_swiglu", ms, flops
+
+
+def run_coda(a):
+    import torch
+    import torch.distributed as dist
+    kind, s, bwd = WORKLOADS[a.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py: no CUDA device (the library has no CPU path)")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    host, dev = _setup(kind, s, bwd, device)
+    step, outs, launches, result_keys, ws = _make_step(kind, s, bwd, dev)
+    flops = _flops(kind, s, bwd)
+
+    for _ in range(max(a.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    st = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        e0.record(st)
+        for _ in range(a.steps):
+            step()
+        e1.record(st)
+        torch.cuda.synchronize()
+        barrier()
+    ms_total = e0.elapsed_time(e1)
+    status, detail = ws.query()
+    if status != 0:
+        raise SystemExit(f"bench.py: device status {status} detail {detail:#x}")
+    t = torch.tensor([ms_total], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    value = flops * a.steps * world / (ms_max / 1e3) / 1e12
+
+    # Dominant kernel alone (roofline).
+    peaks, peaks_src = _peaks()
+    kname, k_ms, k_flops = _dominant_kernel(kind, s, dev, outs)
+    achieved = k_flops / (k_ms / 1e3) / 1e12
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    roofline = {"bound": "tensor", "kernel": kname, "achieved": round(achieved, 1), "peak": peak,
+                "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                "traffic": _recorded_traffic(kname, a.workload), "peak_source": f"{peaks_src} burst bf16",
+                "launch_ms": round(k_ms, 4)}
+
+    # End to end through the public API with host buffers (pinned), copies inside the timed region.
+    e2e = None
+    if not a.no_e2e:
+        pin_in = {k: v.pin_memory() for k, v in host.items()}
+        pin_out = {k: torch.empty(outs[k].shape, dtype=outs[k].dtype, pin_memory=True) for k in result_keys}
+        h2d = sum(v.numel() * v.element_size() for v in pin_in.values())
+        d2h = sum(v.numel() * v.element_size() for v in pin_out.values())
+
+        def e2e_step():
+            for k, v in pin_in.items():
+                dev[k].copy_(v, non_blocking=True)
+            step()
+            for k in result_keys:
+                pin_out[k].copy_(outs[k], non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        n_e2e = max(3, min(a.steps, 10))
+        barrier()
+        e0.record(st)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(st)
+        torch.cuda.synchronize()
+        barrier()
+        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=device)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e = {"value": round(flops * n_e2e * world / (float(te.item()) / 1e3) / 1e12, 2), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": n_e2e}
+
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        cpu = cpu_baseline(kind, s, bwd)
+
+    if rank == 0:
+        frac_step = value / world / float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+        line = {
+            "metric": METRIC,
+            "value": round(value, 2),
+            "unit": "TFLOP/s",
+            "n_gpus": world,
+            "steps": a.steps,
+            "warmup": max(a.warmup, 3),
+            "ms_per_step": round(ms_max / a.steps, 4),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic",
+            "config": {**_describe(a.workload, kind, s, bwd), "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2 (step working set > 1 GB), no flush",
+                       "flops_per_step": flops, "frac_of_sustained_bf16_peak": round(frac_step, 4)},
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches * a.steps,
+            "clocks": clk.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def run_reference(a):
+    """The reference arm: the fp64 CPU oracle on the host cores, bounded samples of the workload."""
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    kind, s, bwd = WORKLOADS[a.workload]
+    inputs = _oracle_inputs(kind, s)
+    probe = min(64, s["M"])
+    t0 = time.perf_counter()
+    _oracle_step(kind, s, bwd, inputs, probe)
+    rate = _flops(kind, dict(s, M=probe), bwd) / max(time.perf_counter() - t0, 1e-3)
+    # Each step a sample sized for about 2 s so the whole run stays within a few minutes.
+    rows = max(probe, min(s["M"], int(2.0 * rate / _flops(kind, dict(s, M=1), bwd))))
+    for _ in range(a.warmup):
+        _oracle_step(kind, s, bwd, inputs, rows)
+    t0 = time.perf_counter()
+    for _ in range(a.steps):
+        _oracle_step(kind, s, bwd, inputs, rows)
+    dt = time.perf_counter() - t0
+    fl = _flops(kind, dict(s, M=rows), bwd)
+    value = fl * a.steps / dt / 1e12
+    sample = (f"fp64 numpy oracle, unfused textbook {'fwd+bwd' if bwd else 'fwd'} on the first {rows} of "
+              f"{s['M']} tokens with the full weights per step")
+    line = {
+        "metric": METRIC, "value": round(value, 4), "unit": "TFLOP/s", "n_gpus": world, "steps": a.steps,
+        "warmup": a.warmup, "ms_per_step": round(dt / a.steps * 1e3, 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {**_describe(a.workload, kind, s, bwd), "parallelism": "host cores", "sample_rows": rows},
+        "cpu_baseline": {"value": round(value, 4), "unit": "TFLOP/s", "cores": _blas_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    a = _args()
+    if a.impl == "reference":
+        run_reference(a)
+    else:
+        run_coda(a)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,292 @@
+"""Python binding of the C-ABI library (argument marshalling only).
+
+Every step of the path runs in the CUDA kernels of ``libcoda.so``; this module
+checks tensor dtypes/devices/contiguity, allocates outputs and the workspace
+with torch (device memory and streams are all torch is used for), and passes
+raw device pointers plus ``torch.cuda.current_stream()`` to the C entry points
+of the same names.  There is no CPU fallback: if the library is missing or the
+device is not sm_100, calls raise.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+from .build import LIB_PATH
+
+_c_void_p = ctypes.c_void_p
+_c_int = ctypes.c_int
+_c_size_t = ctypes.c_size_t
+_c_float = ctypes.c_float
+
+CODA_ERR_DEVICE_TIMEOUT = 7
+
+
+class CodaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = int(status)
+        super().__init__(f"{where}: {_status_string(status)} (status {status})")
+
+
+_lib = None
+_lib_lock = threading.Lock()
+
+
+def library() -> ctypes.CDLL:
+    """Load libcoda.so (built in-tree by gemm_epilogue_fusion_tmem_b200.build)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    with _lib_lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"CUDA library not built ({LIB_PATH}); run `python -m gemm_epilogue_fusion_tmem_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        P, I, S, F = _c_void_p, _c_int, _c_size_t, _c_float
+        sig = {
+            "coda_status_string": (ctypes.c_char_p, [I]),
+            "coda_version": (I, []),
+            "coda_status_clear": (I, [P, P]),
+            "coda_status_query": (I, [P, P, ctypes.POINTER(ctypes.c_uint32)]),
+            "coda_set_wait_limit_ns": (None, [ctypes.c_uint64]),
+            "coda_gemm_workspace_bytes": (S, []),
+            "coda_gemm": (I, [P, P, P, I, I, I, I, I, P, S, P]),
+            "coda_fold_gain": (I, [P, P, P, I, I, P]),
+            "coda_gemm_swiglu": (I, [P, P, P, P, P, I, I, I, P, S, P]),
+            "coda_grg_fwd_workspace_bytes": (S, [I, I, I, I, I]),
+            "coda_grg_fwd": (I, [P, P, P, P, P, P, P, P, P, P, I, I, I, I, F, P, S, P]),
+            "coda_grg_bwd_workspace_bytes": (S, [I, I, I, I]),
+            "coda_grg_bwd": (I, [P, P, P, P, P, P, P, P, P, P, P, P, P, P, I, I, I, I, P, S, P]),
+            "coda_swiglu_fwd_workspace_bytes": (S, [I, I, I]),
+            "coda_swiglu_fwd": (I, [P, P, P, P, P, P, I, I, I, P, S, P]),
+            "coda_swiglu_bwd_workspace_bytes": (S, [I, I, I]),
+            "coda_swiglu_bwd": (I, [P, P, P, P, P, P, P, P, P, I, I, I, P, S, P]),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+        return lib
+
+
+def _status_string(status: int) -> str:
+    try:
+        return library().coda_status_string(int(status)).decode()
+    except Exception:  # pragma: no cover - only when the library cannot load
+        return "unknown"
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise CodaError(status, where)
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _req(t: torch.Tensor, name: str, dtype=torch.bfloat16, shape=None) -> torch.Tensor:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (no CPU path exists)")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t
+
+
+# ------------------------------------------------------------------ workspace
+
+class Workspace:
+    """A caller-owned device workspace whose first 256 bytes are the status word."""
+
+    def __init__(self, nbytes: int, device=None):
+        self.buf = torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device or "cuda")
+
+    @property
+    def nbytes(self) -> int:
+        return self.buf.numel()
+
+    def ptr(self):
+        return ctypes.c_void_p(self.buf.data_ptr())
+
+    def clear(self) -> None:
+        _check(library().coda_status_clear(self.ptr(), _stream()), "coda_status_clear")
+
+    def query(self) -> tuple[int, int]:
+        """Synchronise the current stream and return (status, detail)."""
+        detail = ctypes.c_uint32(0)
+        st = library().coda_status_query(self.ptr(), _stream(), ctypes.byref(detail))
+        return int(st), int(detail.value)
+
+
+_ws_cache: dict = {}
+
+
+def workspace(nbytes: int, device=None) -> Workspace:
+    """Per-device cached workspace grown on demand (zeroed when (re)allocated)."""
+    dev = torch.device(device or "cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    ws = _ws_cache.get(dev)
+    if ws is None or ws.nbytes < nbytes:
+        ws = Workspace(nbytes, dev)
+        _ws_cache[dev] = ws
+    return ws
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    library().coda_set_wait_limit_ns(int(ns))
+
+
+# ------------------------------------------------------------------ entry points
+
+def gemm(A: torch.Tensor, B: torch.Tensor, M: int, N: int, K: int, a_mn_major: bool = False,
+         b_mn_major: bool = False, out: torch.Tensor | None = None, ws: Workspace | None = None) -> torch.Tensor:
+    """C[M,N] = op(A) op(B)^T (bf16 out, fp32 accumulate); see coda_gemm in include/coda.h."""
+    lib = library()
+    _req(A, "A", shape=(K, M) if a_mn_major else (M, K))
+    _req(B, "B", shape=(K, N) if b_mn_major else (N, K))
+    C = out if out is not None else torch.empty(M, N, dtype=torch.bfloat16, device=A.device)
+    _req(C, "C", shape=(M, N))
+    ws = ws or workspace(lib.coda_gemm_workspace_bytes(), A.device)
+    _check(lib.coda_gemm(_ptr(A), _ptr(B), _ptr(C), M, N, K, int(a_mn_major), int(b_mn_major),
+                         ws.ptr(), ws.nbytes, _stream()), "coda_gemm")
+    return C
+
+
+def gemm_swiglu(A, Wgu, r=None, save_ab: bool = True, out: dict | None = None,
+                ws: Workspace | None = None) -> dict:
+    """Y = silu(r*(A Wgu^T)_gate) * (r*(A Wgu^T)_up), AB = [a | b]; see coda_gemm_swiglu."""
+    lib = library()
+    M, K = A.shape
+    F = Wgu.shape[0] // 2
+    _req(A, "A"), _req(Wgu, "Wgu", shape=(2 * F, K))
+    if r is not None:
+        _req(r, "r", torch.float32, (M,))
+    o = dict(out or {})
+    o.setdefault("Y", torch.empty(M, F, dtype=torch.bfloat16, device=A.device))
+    if save_ab:
+        o.setdefault("AB", torch.empty(M, 2 * F, dtype=torch.bfloat16, device=A.device))
+    ws = ws or workspace(lib.coda_gemm_workspace_bytes(), A.device)
+    _check(lib.coda_gemm_swiglu(_ptr(A), _ptr(Wgu), _ptr(r), _ptr(o["Y"]), _ptr(o.get("AB") if save_ab else None),
+                                M, K, F, ws.ptr(), ws.nbytes, _stream()), "coda_gemm_swiglu")
+    return o
+
+
+def fold_gain(W2: torch.Tensor, g: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """W2g = W2 * g (per column), bf16; see coda_fold_gain."""
+    N, d = W2.shape
+    _req(W2, "W2")
+    _req(g, "g", shape=(d,))
+    W2g = out if out is not None else torch.empty_like(W2)
+    _req(W2g, "W2g", shape=(N, d))
+    _check(library().coda_fold_gain(_ptr(W2), _ptr(g), _ptr(W2g), d, N, _stream()), "coda_fold_gain")
+    return W2g
+
+
+def grg_fwd(X, W1, R, g, W2, eps: float, W2g=None, save_ab: bool = True, out: dict | None = None,
+            ws: Workspace | None = None) -> dict:
+    """Fused GEMM-Residual-PartialRMS-GEMM-SwiGLU forward; returns H, r, Y, AB."""
+    lib = library()
+    M, K = X.shape
+    d = W1.shape[0]
+    N = W2.shape[0]
+    F = N // 2
+    _req(X, "X"), _req(W1, "W1", shape=(d, K)), _req(R, "R", shape=(M, d))
+    _req(g, "g", shape=(d,)), _req(W2, "W2", shape=(N, d))
+    if W2g is not None:
+        _req(W2g, "W2g", shape=(N, d))
+    o = dict(out or {})
+    dev = X.device
+    o.setdefault("H", torch.empty(M, d, dtype=torch.bfloat16, device=dev))
+    o.setdefault("r", torch.empty(M, dtype=torch.float32, device=dev))
+    o.setdefault("Y", torch.empty(M, F, dtype=torch.bfloat16, device=dev))
+    if save_ab:
+        o.setdefault("AB", torch.empty(M, N, dtype=torch.bfloat16, device=dev))
+    _req(o["H"], "H", shape=(M, d)), _req(o["r"], "r", torch.float32, (M,)), _req(o["Y"], "Y", shape=(M, F))
+    AB = o.get("AB") if save_ab else None
+    if AB is not None:
+        _req(AB, "AB", shape=(M, N))
+    need = lib.coda_grg_fwd_workspace_bytes(M, K, d, N, int(W2g is not None))
+    ws = ws or workspace(need, dev)
+    _check(lib.coda_grg_fwd(_ptr(X), _ptr(W1), _ptr(R), _ptr(g), _ptr(W2), _ptr(W2g), _ptr(o["H"]),
+                            _ptr(o["r"]), _ptr(o["Y"]), _ptr(AB), M, K, d, N, float(eps),
+                            ws.ptr(), ws.nbytes, _stream()), "coda_grg_fwd")
+    return o
+
+
+def grg_bwd(dY, X, W1, H, r, AB, g, W2, dH_in=None, out: dict | None = None, ws: Workspace | None = None) -> dict:
+    """Fused backward of the block; returns dX, dR, dW1, dW2, dg."""
+    lib = library()
+    M, K = X.shape
+    d = W1.shape[0]
+    N = W2.shape[0]
+    F = N // 2
+    _req(dY, "dY", shape=(M, F)), _req(X, "X"), _req(W1, "W1", shape=(d, K)), _req(H, "H", shape=(M, d))
+    _req(r, "r", torch.float32, (M,)), _req(AB, "AB", shape=(M, N)), _req(g, "g", shape=(d,))
+    _req(W2, "W2", shape=(N, d))
+    if dH_in is not None:
+        _req(dH_in, "dH_in", shape=(M, d))
+    o = dict(out or {})
+    dev = X.device
+    o.setdefault("dX", torch.empty(M, K, dtype=torch.bfloat16, device=dev))
+    o.setdefault("dR", torch.empty(M, d, dtype=torch.bfloat16, device=dev))
+    o.setdefault("dW1", torch.empty(d, K, dtype=torch.bfloat16, device=dev))
+    o.setdefault("dW2", torch.empty(N, d, dtype=torch.bfloat16, device=dev))
+    o.setdefault("dg", torch.empty(d, dtype=torch.float32, device=dev))
+    ws = ws or workspace(lib.coda_grg_bwd_workspace_bytes(M, K, d, N), dev)
+    _check(lib.coda_grg_bwd(_ptr(dY), _ptr(dH_in), _ptr(X), _ptr(W1), _ptr(H), _ptr(r), _ptr(AB), _ptr(g),
+                            _ptr(W2), _ptr(o["dX"]), _ptr(o["dR"]), _ptr(o["dW1"]), _ptr(o["dW2"]), _ptr(o["dg"]),
+                            M, K, d, N, ws.ptr(), ws.nbytes, _stream()), "coda_grg_bwd")
+    return o
+
+
+def swiglu_fwd(X, Wgu, Wdown, save_ab: bool = True, out: dict | None = None, ws: Workspace | None = None) -> dict:
+    """SwiGLU MLP forward; returns Y, AB, Out."""
+    lib = library()
+    M, d = X.shape
+    F = Wgu.shape[0] // 2
+    _req(X, "X"), _req(Wgu, "Wgu", shape=(2 * F, d)), _req(Wdown, "Wdown", shape=(d, F))
+    o = dict(out or {})
+    dev = X.device
+    o.setdefault("Y", torch.empty(M, F, dtype=torch.bfloat16, device=dev))
+    if save_ab:
+        o.setdefault("AB", torch.empty(M, 2 * F, dtype=torch.bfloat16, device=dev))
+    o.setdefault("Out", torch.empty(M, d, dtype=torch.bfloat16, device=dev))
+    ws = ws or workspace(lib.coda_swiglu_fwd_workspace_bytes(M, d, F), dev)
+    _check(lib.coda_swiglu_fwd(_ptr(X), _ptr(Wgu), _ptr(Wdown), _ptr(o["Y"]), _ptr(o.get("AB") if save_ab else None),
+                               _ptr(o["Out"]), M, d, F, ws.ptr(), ws.nbytes, _stream()), "coda_swiglu_fwd")
+    return o
+
+
+def swiglu_bwd(dOut, X, Wgu, Wdown, Y, AB, out: dict | None = None, ws: Workspace | None = None) -> dict:
+    """SwiGLU MLP backward; returns dX, dWgu, dWdown."""
+    lib = library()
+    M, d = X.shape
+    F = Wgu.shape[0] // 2
+    _req(dOut, "dOut", shape=(M, d)), _req(X, "X"), _req(Wgu, "Wgu", shape=(2 * F, d))
+    _req(Wdown, "Wdown", shape=(d, F)), _req(Y, "Y", shape=(M, F)), _req(AB, "AB", shape=(M, 2 * F))
+    o = dict(out or {})
+    dev = X.device
+    o.setdefault("dX", torch.empty(M, d, dtype=torch.bfloat16, device=dev))
+    o.setdefault("dWgu", torch.empty(2 * F, d, dtype=torch.bfloat16, device=dev))
+    o.setdefault("dWdown", torch.empty(d, F, dtype=torch.bfloat16, device=dev))
+    ws = ws or workspace(lib.coda_swiglu_bwd_workspace_bytes(M, d, F), dev)
+    _check(lib.coda_swiglu_bwd(_ptr(dOut), _ptr(X), _ptr(Wgu), _ptr(Wdown), _ptr(Y), _ptr(AB), _ptr(o["dX"]),
+                               _ptr(o["dWgu"]), _ptr(o["dWdown"]), M, d, F, ws.ptr(), ws.nbytes, _stream()),
+           "coda_swiglu_bwd")
+    return o

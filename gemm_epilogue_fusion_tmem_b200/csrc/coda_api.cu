@@ -1,0 +1,479 @@
+// C-ABI entry points (include/coda.h): argument validation, workspace carving,
+// TMA tensor-map encoding and the launch sequence of each fused pass.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+
+#include "coda.h"
+#include "coda_aux.cuh"
+#include "coda_gemm.cuh"
+
+namespace coda {
+namespace {
+
+constexpr size_t kStatusBytes = 256;
+std::atomic<unsigned long long> g_wait_limit_ns{4000000000ull};
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline int cdiv(long long a, long long b) { return (int)((a + b - 1) / b); }
+
+// ------------------------------------------------------------------ device checks
+
+struct DevInfo {
+  int num_sms = 0;
+  int major = 0;
+  bool smem_set[16] = {};
+};
+DevInfo g_dev[64];
+
+coda_status current_device(int& dev) {
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return CODA_ERR_CUDA;
+  DevInfo& di = g_dev[dev];
+  if (di.num_sms == 0) {
+    int sms = 0, major = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return CODA_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return CODA_ERR_CUDA;
+    di.major = major;
+    di.num_sms = sms;
+  }
+  if (di.major != 10) return CODA_ERR_NO_SM100;
+  return CODA_OK;
+}
+
+// ------------------------------------------------------------------ tensor maps
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// Row-major bf16 matrix [rows][cols] (cols contiguous), 128-byte swizzled
+// boxes of box_cols x box_rows; out-of-range elements load as zero.
+bool make_tmap(CUtensorMap* m, const void* base, long long rows, long long cols, int box_cols, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Operand with logical shape [mn, k].  K-major storage is [mn][k]; MN-major
+// storage is [k][mn].  box_mn is the tile extent along mn for K-major maps.
+bool make_operand_map(CUtensorMap* m, const void* base, long long mn, long long k, bool mn_major, int box_mn) {
+  if (!mn_major) return make_tmap(m, base, mn, k, BK, box_mn);
+  return make_tmap(m, base, k, mn, 64, BK);
+}
+
+// ------------------------------------------------------------------ GEMM launch
+
+template <int EPI, bool A_MN, bool B_MN>
+coda_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, GemmParams p, cudaStream_t s) {
+  int dev = 0;
+  coda_status st = current_device(dev);
+  if (st != CODA_OK) return st;
+  auto kern = gemm_tc_kernel<EPI, A_MN, B_MN>;
+  const int slot = EPI * 4 + (A_MN ? 2 : 0) + (B_MN ? 1 : 0);
+  if (!g_dev[dev].smem_set[slot]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES) != cudaSuccess)
+      return CODA_ERR_CUDA;
+    g_dev[dev].smem_set[slot] = true;
+  }
+  p.kernel_id = (uint32_t)(slot + 1);
+  p.wait_limit_ns = g_wait_limit_ns.load();
+  const int tiles = p.num_m_tiles * p.num_n_tiles;
+  const int grid = std::min(tiles, g_dev[dev].num_sms);
+  if (grid <= 0) return CODA_OK;
+  kern<<<grid, NUM_THREADS, GEMM_SMEM_BYTES, s>>>(ta, tb, p);
+  return cudaPeekAtLastError() == cudaSuccess ? CODA_OK : CODA_ERR_CUDA;
+}
+
+GemmParams base_params(int M, int N, int K, int tile_n, void* ws) {
+  GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.num_m_tiles = cdiv(M, BM);
+  p.num_n_tiles = cdiv(N, tile_n);
+  p.k_blocks = cdiv(K, BK);
+  p.status = static_cast<uint32_t*>(ws);
+  return p;
+}
+
+inline __nv_bfloat16* bf(void* p) { return static_cast<__nv_bfloat16*>(p); }
+inline const __nv_bfloat16* cbf(const void* p) { return static_cast<const __nv_bfloat16*>(p); }
+
+// Plain C = op(A) op(B)^T with the EPI_STORE epilogue (optional column scale).
+coda_status gemm_store(const void* A, const void* B, void* C, int M, int N, int K, bool a_mn, bool b_mn,
+                       const void* colscale, void* ws, cudaStream_t s) {
+  CUtensorMap ta, tb;
+  if (!make_operand_map(&ta, A, M, K, a_mn, BM) || !make_operand_map(&tb, B, N, K, b_mn, BN))
+    return CODA_ERR_CUDA;
+  GemmParams p = base_params(M, N, K, BN, ws);
+  p.out = bf(C);
+  p.ldo = N;
+  p.colvec = cbf(colscale);
+  if (!a_mn && !b_mn) return launch_gemm<EPI_STORE, false, false>(ta, tb, p, s);
+  if (!a_mn && b_mn) return launch_gemm<EPI_STORE, false, true>(ta, tb, p, s);
+  if (a_mn && b_mn) return launch_gemm<EPI_STORE, true, true>(ta, tb, p, s);
+  return launch_gemm<EPI_STORE, true, false>(ta, tb, p, s);
+}
+
+coda_status launch_status(cudaError_t e) { return e == cudaSuccess ? CODA_OK : CODA_ERR_CUDA; }
+
+// Gate/up GEMM with the row-scale + SwiGLU epilogue (r may be null).
+coda_status gemm_swiglu(const void* A, const void* Wgu, const float* r, void* Y, void* AB, int M, int K, int F,
+                        void* ws, cudaStream_t s) {
+  CUtensorMap ta, tb;
+  if (!make_operand_map(&ta, A, M, K, false, BM) || !make_operand_map(&tb, Wgu, 2LL * F, K, false, BN / 2))
+    return CODA_ERR_CUDA;
+  GemmParams p = base_params(M, F, K, BN / 2, ws);
+  p.split = F;
+  p.out = bf(Y);
+  p.ldo = F;
+  p.out2 = bf(AB);
+  p.ldo2 = 2 * F;
+  p.rowvec = r;
+  return launch_gemm<EPI_SWIGLU, false, false>(ta, tb, p, s);
+}
+
+}  // namespace
+}  // namespace coda
+
+using namespace coda;
+
+#define CODA_TRY(expr)                 \
+  do {                                 \
+    coda_status _s = (expr);           \
+    if (_s != CODA_OK) return _s;      \
+  } while (0)
+
+extern "C" {
+
+const char* coda_status_string(int s) {
+  switch (s) {
+    case CODA_OK: return "ok";
+    case CODA_ERR_INVALID_ARG: return "invalid argument";
+    case CODA_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case CODA_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case CODA_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case CODA_ERR_NO_SM100: return "device is not sm_100 (B200)";
+    case CODA_ERR_CUDA: return "CUDA error";
+    case CODA_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int coda_version(void) { return 100; }
+
+void coda_set_wait_limit_ns(uint64_t ns) {
+  ns = std::max<uint64_t>(ns, 1000ull);
+  ns = std::min<uint64_t>(ns, 60000000000ull);
+  g_wait_limit_ns.store(ns);
+}
+
+coda_status coda_status_clear(void* ws, void* stream) {
+  if (ws == nullptr) return CODA_ERR_INVALID_ARG;
+  return launch_status(cudaMemsetAsync(ws, 0, kStatusBytes, static_cast<cudaStream_t>(stream)));
+}
+
+coda_status coda_status_query(const void* ws, void* stream, uint32_t* detail) {
+  if (ws == nullptr) return CODA_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return CODA_ERR_CUDA;
+  uint32_t w[2] = {0, 0};
+  if (cudaMemcpy(w, ws, sizeof(w), cudaMemcpyDeviceToHost) != cudaSuccess) return CODA_ERR_CUDA;
+  if (detail != nullptr) *detail = w[1];
+  return static_cast<coda_status>(w[0]);
+}
+
+// ------------------------------------------------------------------ plain GEMM
+
+size_t coda_gemm_workspace_bytes(void) { return kStatusBytes; }
+
+coda_status coda_gemm(const void* A, const void* B, void* C, int M, int N, int K, int a_mn_major, int b_mn_major,
+                      void* ws, size_t ws_bytes, void* stream) {
+  if (!A || !B || !C || !ws) return CODA_ERR_INVALID_ARG;
+  if (M < 1 || N < 1 || K < 1) return CODA_ERR_INVALID_ARG;
+  if (N % 32 != 0) return CODA_ERR_UNSUPPORTED_SHAPE;
+  if ((a_mn_major ? M : K) % 8 != 0 || (b_mn_major ? N : K) % 8 != 0) return CODA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(C) || !aligned16(ws)) return CODA_ERR_MISALIGNED;
+  if (ws_bytes < coda_gemm_workspace_bytes()) return CODA_ERR_WORKSPACE_TOO_SMALL;
+  int dev;
+  CODA_TRY(current_device(dev));
+  return gemm_store(A, B, C, M, N, K, a_mn_major != 0, b_mn_major != 0, nullptr, ws,
+                    static_cast<cudaStream_t>(stream));
+}
+
+coda_status coda_gemm_swiglu(const void* A, const void* Wgu, const float* r_or_null, void* Y, void* AB_or_null,
+                             int M, int K, int F, void* ws, size_t ws_bytes, void* stream) {
+  if (!A || !Wgu || !Y || !ws) return CODA_ERR_INVALID_ARG;
+  if (M < 1 || K < 1 || F < 1) return CODA_ERR_INVALID_ARG;
+  if (K % 64 != 0 || F % 64 != 0) return CODA_ERR_UNSUPPORTED_SHAPE;
+  const void* ptrs[] = {A, Wgu, r_or_null, Y, AB_or_null, ws};
+  for (const void* q : ptrs)
+    if (q && !aligned16(q)) return CODA_ERR_MISALIGNED;
+  if (ws_bytes < coda_gemm_workspace_bytes()) return CODA_ERR_WORKSPACE_TOO_SMALL;
+  int dev;
+  CODA_TRY(current_device(dev));
+  return gemm_swiglu(A, Wgu, r_or_null, Y, AB_or_null, M, K, F, ws, static_cast<cudaStream_t>(stream));
+}
+
+// ------------------------------------------------------------------ gain fold
+
+coda_status coda_fold_gain(const void* W2, const void* g, void* W2g, int d, int N, void* stream) {
+  if (!W2 || !g || !W2g) return CODA_ERR_INVALID_ARG;
+  if (d < 1 || N < 1) return CODA_ERR_INVALID_ARG;
+  if (d % 8 != 0) return CODA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(W2) || !aligned16(g) || !aligned16(W2g)) return CODA_ERR_MISALIGNED;
+  int dev;
+  CODA_TRY(current_device(dev));
+  const long long nv = (long long)N * d / 8;
+  const int grid = (int)std::min<long long>(cdiv(nv, 256), (long long)g_dev[dev].num_sms * 8);
+  fold_gain_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(cbf(W2), cbf(g), bf(W2g), d, nv);
+  return launch_status(cudaPeekAtLastError());
+}
+
+// ------------------------------------------------------------------ GRG forward
+
+namespace {
+constexpr int kRmsTile = BN;  // columns per partial sum of squares
+struct FwdWs {
+  size_t p_off, w2g_off, total;
+};
+FwdWs fwd_ws(int M, int d, int N, bool prefolded) {
+  FwdWs w;
+  const int T = cdiv(d, kRmsTile);
+  w.p_off = kStatusBytes;
+  w.w2g_off = align_up(w.p_off + (size_t)M * T * 4, 256);
+  w.total = w.w2g_off + (prefolded ? 0 : align_up((size_t)N * d * 2, 256));
+  return w;
+}
+
+coda_status check_grg_shapes(int M, int K, int d, int N) {
+  if (M < 1 || K < 1 || d < 1 || N < 2) return CODA_ERR_INVALID_ARG;
+  if (K % 64 != 0 || d % 64 != 0 || N % 128 != 0) return CODA_ERR_UNSUPPORTED_SHAPE;
+  return CODA_OK;
+}
+}  // namespace
+
+size_t coda_grg_fwd_workspace_bytes(int M, int K, int d, int N, int prefolded) {
+  (void)K;
+  if (M < 1 || d < 1 || N < 1) return kStatusBytes;
+  return fwd_ws(M, d, N, prefolded != 0).total;
+}
+
+coda_status coda_grg_fwd(const void* X, const void* W1, const void* R, const void* g, const void* W2,
+                         const void* W2g_or_null, void* H, float* r, void* Y, void* AB_or_null, int M, int K, int d,
+                         int N, float eps, void* ws, size_t ws_bytes, void* stream) {
+  if (!X || !W1 || !R || !H || !r || !Y || !ws) return CODA_ERR_INVALID_ARG;
+  if (W2g_or_null == nullptr && (!g || !W2)) return CODA_ERR_INVALID_ARG;
+  if (!(eps > 0.f)) return CODA_ERR_INVALID_ARG;
+  CODA_TRY(check_grg_shapes(M, K, d, N));
+  const void* ptrs[] = {X, W1, R, g, W2, W2g_or_null, H, r, Y, AB_or_null, ws};
+  for (const void* q : ptrs)
+    if (q && !aligned16(q)) return CODA_ERR_MISALIGNED;
+  const bool prefolded = W2g_or_null != nullptr;
+  const FwdWs w = fwd_ws(M, d, N, prefolded);
+  if (ws_bytes < w.total) return CODA_ERR_WORKSPACE_TOO_SMALL;
+  int dev;
+  CODA_TRY(current_device(dev));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  float* P = reinterpret_cast<float*>(wsb + w.p_off);
+  const int T = cdiv(d, kRmsTile);
+  const int F = N / 2;
+
+  // Gain fold (skipped when the caller supplies diag(g)-scaled W2).
+  const void* W2g = W2g_or_null;
+  if (!prefolded) {
+    W2g = wsb + w.w2g_off;
+    CODA_TRY(coda_fold_gain(W2, g, const_cast<void*>(W2g), d, N, stream));
+  }
+
+  // GEMM1 + residual + partial sums of squares.
+  {
+    CUtensorMap ta, tb;
+    if (!make_operand_map(&ta, X, M, K, false, BM) || !make_operand_map(&tb, W1, d, K, false, BN))
+      return CODA_ERR_CUDA;
+    GemmParams p = base_params(M, d, K, BN, ws);
+    p.out = bf(H);
+    p.ldo = d;
+    p.in0 = cbf(R);
+    p.ld_in0 = d;
+    p.part = P;
+    p.ld_part = T;
+    CODA_TRY((launch_gemm<EPI_RESID_RMS, false, false>(ta, tb, p, s)));
+  }
+  // Row reduce -> r.
+  rms_rowreduce_kernel<<<cdiv(M, 256), 256, 0, s>>>(P, T, r, M, 1.0f / (float)d, eps);
+  CODA_TRY(launch_status(cudaPeekAtLastError()));
+  // GEMM2 (gate|up) + r scaling + SwiGLU.
+  CODA_TRY(gemm_swiglu(H, W2g, r, Y, AB_or_null, M, d, F, ws, s));
+  return CODA_OK;
+}
+
+// ------------------------------------------------------------------ GRG backward
+
+namespace {
+struct BwdWs {
+  size_t dap_off, c_off, pg_off, total;
+  int pg_rows;
+};
+BwdWs bwd_ws(int M, int d, int N) {
+  BwdWs w;
+  w.dap_off = kStatusBytes;
+  w.c_off = align_up(w.dap_off + (size_t)M * N * 2, 256);
+  w.pg_off = align_up(w.c_off + (size_t)M * 4, 256);
+  w.pg_rows = cdiv(M, BM) * 4;
+  w.total = align_up(w.pg_off + (size_t)w.pg_rows * d * 4, 256);
+  return w;
+}
+}  // namespace
+
+size_t coda_grg_bwd_workspace_bytes(int M, int K, int d, int N) {
+  (void)K;
+  if (M < 1 || d < 1 || N < 1) return kStatusBytes;
+  return bwd_ws(M, d, N).total;
+}
+
+coda_status coda_grg_bwd(const void* dY, const void* dH_in_or_null, const void* X, const void* W1, const void* H,
+                         const float* r, const void* AB, const void* g, const void* W2, void* dX, void* dR,
+                         void* dW1, void* dW2, float* dg, int M, int K, int d, int N, void* ws, size_t ws_bytes,
+                         void* stream) {
+  if (!dY || !X || !W1 || !H || !r || !AB || !g || !W2 || !dX || !dR || !dW1 || !dW2 || !dg || !ws)
+    return CODA_ERR_INVALID_ARG;
+  CODA_TRY(check_grg_shapes(M, K, d, N));
+  const void* ptrs[] = {dY, dH_in_or_null, X, W1, H, r, AB, g, W2, dX, dR, dW1, dW2, dg, ws};
+  for (const void* q : ptrs)
+    if (q && !aligned16(q)) return CODA_ERR_MISALIGNED;
+  const BwdWs w = bwd_ws(M, d, N);
+  if (ws_bytes < w.total) return CODA_ERR_WORKSPACE_TOO_SMALL;
+  int dev;
+  CODA_TRY(current_device(dev));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  __nv_bfloat16* dAp = reinterpret_cast<__nv_bfloat16*>(wsb + w.dap_off);
+  float* cvec = reinterpret_cast<float*>(wsb + w.c_off);
+  float* Pg = reinterpret_cast<float*>(wsb + w.pg_off);
+  const int F = N / 2;
+
+  // SwiGLU backward + RMSNorm row statistic.
+  swiglu_bwd_rowstat_kernel<<<M, ROWSTAT_THREADS, 0, s>>>(cbf(dY), cbf(AB), r, dAp, cvec, F, 1.0f / (float)d);
+  CODA_TRY(launch_status(cudaPeekAtLastError()));
+  // dn GEMM: dR = g * (dA' W2) - c * H (+ dH_in), with dg column partials.
+  {
+    CUtensorMap ta, tb;
+    if (!make_operand_map(&ta, dAp, M, N, false, BM) || !make_operand_map(&tb, W2, d, N, true, BN))
+      return CODA_ERR_CUDA;
+    GemmParams p = base_params(M, d, N, BN, ws);
+    p.out = bf(dR);
+    p.ldo = d;
+    p.in0 = cbf(H);
+    p.ld_in0 = d;
+    p.in1 = cbf(dH_in_or_null);
+    p.colvec = cbf(g);
+    p.rowvec = cvec;
+    p.part = Pg;
+    p.ld_part = d;
+    CODA_TRY((launch_gemm<EPI_DN, false, true>(ta, tb, p, s)));
+  }
+  col_reduce_kernel<<<cdiv(d, 256), 256, 0, s>>>(Pg, w.pg_rows, d, dg);
+  CODA_TRY(launch_status(cudaPeekAtLastError()));
+  // dW2 = g * (dA'^T H).
+  CODA_TRY(gemm_store(dAp, H, dW2, N, d, M, true, true, g, ws, s));
+  // dX = dH W1;  dW1 = dH^T X.
+  CODA_TRY(gemm_store(dR, W1, dX, M, K, d, false, true, nullptr, ws, s));
+  CODA_TRY(gemm_store(dR, X, dW1, d, K, M, true, true, nullptr, ws, s));
+  return CODA_OK;
+}
+
+// ------------------------------------------------------------------ SwiGLU MLP
+
+namespace {
+coda_status check_swiglu_shapes(int M, int d, int F) {
+  if (M < 1 || d < 1 || F < 1) return CODA_ERR_INVALID_ARG;
+  if (d % 64 != 0 || F % 64 != 0) return CODA_ERR_UNSUPPORTED_SHAPE;
+  return CODA_OK;
+}
+}  // namespace
+
+size_t coda_swiglu_fwd_workspace_bytes(int M, int d, int F) {
+  (void)M, (void)d, (void)F;
+  return kStatusBytes;
+}
+
+coda_status coda_swiglu_fwd(const void* X, const void* Wgu, const void* Wdown, void* Y, void* AB_or_null,
+                            void* Out, int M, int d, int F, void* ws, size_t ws_bytes, void* stream) {
+  if (!X || !Wgu || !Wdown || !Y || !Out || !ws) return CODA_ERR_INVALID_ARG;
+  CODA_TRY(check_swiglu_shapes(M, d, F));
+  const void* ptrs[] = {X, Wgu, Wdown, Y, AB_or_null, Out, ws};
+  for (const void* q : ptrs)
+    if (q && !aligned16(q)) return CODA_ERR_MISALIGNED;
+  if (ws_bytes < coda_swiglu_fwd_workspace_bytes(M, d, F)) return CODA_ERR_WORKSPACE_TOO_SMALL;
+  int dev;
+  CODA_TRY(current_device(dev));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  CODA_TRY(gemm_swiglu(X, Wgu, nullptr, Y, AB_or_null, M, d, F, ws, s));
+  return gemm_store(Y, Wdown, Out, M, d, F, false, false, nullptr, ws, s);
+}
+
+size_t coda_swiglu_bwd_workspace_bytes(int M, int d, int F) {
+  (void)d;
+  if (M < 1 || F < 1) return kStatusBytes;
+  return align_up(kStatusBytes + (size_t)M * 2 * F * 2, 256);
+}
+
+coda_status coda_swiglu_bwd(const void* dOut, const void* X, const void* Wgu, const void* Wdown, const void* Y,
+                            const void* AB, void* dX, void* dWgu, void* dWdown, int M, int d, int F, void* ws,
+                            size_t ws_bytes, void* stream) {
+  if (!dOut || !X || !Wgu || !Wdown || !Y || !AB || !dX || !dWgu || !dWdown || !ws) return CODA_ERR_INVALID_ARG;
+  CODA_TRY(check_swiglu_shapes(M, d, F));
+  const void* ptrs[] = {dOut, X, Wgu, Wdown, Y, AB, dX, dWgu, dWdown, ws};
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return CODA_ERR_MISALIGNED;
+  if (ws_bytes < coda_swiglu_bwd_workspace_bytes(M, d, F)) return CODA_ERR_WORKSPACE_TOO_SMALL;
+  int dev;
+  CODA_TRY(current_device(dev));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  __nv_bfloat16* dA = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(ws) + kStatusBytes);
+  // Down-projection dgrad with the SwiGLU backward in its epilogue.
+  {
+    CUtensorMap ta, tb;
+    if (!make_operand_map(&ta, dOut, M, d, false, BM) || !make_operand_map(&tb, Wdown, F, d, true, BN))
+      return CODA_ERR_CUDA;
+    GemmParams p = base_params(M, F, d, BN, ws);
+    p.split = F;
+    p.out = dA;
+    p.ldo = 2 * F;
+    p.in0 = cbf(AB);
+    p.ld_in0 = 2 * F;
+    CODA_TRY((launch_gemm<EPI_SWIGLU_BWD, false, true>(ta, tb, p, s)));
+  }
+  CODA_TRY(gemm_store(dOut, Y, dWdown, d, F, M, true, true, nullptr, ws, s));
+  CODA_TRY(gemm_store(dA, X, dWgu, 2 * F, d, M, true, true, nullptr, ws, s));
+  CODA_TRY(gemm_store(dA, Wgu, dX, M, d, 2 * F, false, true, nullptr, ws, s));
+  return CODA_OK;
+}
+
+}  // extern "C"

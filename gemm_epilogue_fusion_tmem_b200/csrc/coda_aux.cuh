@@ -1,0 +1,119 @@
+// The light HBM-bound passes around the GEMMs: gain fold, row reduce of the
+// partial sums of squares, SwiGLU backward with its row statistic, and the
+// column reduce of the dg partials.  All use 16-byte vector accesses.
+#pragma once
+
+#include "coda_ptx.cuh"
+
+namespace coda {
+
+// W2g[n, j] = bf16(g[j] * W2[n, j]); 8 elements per thread, d % 8 == 0.
+// The RMSNorm gain as diag(g) folded into the second GEMM's weight (the
+// toolin.ai five-primitive table lists the RMSNorm weight broadcast as a
+// vector-load primitive; folding it once per weight update removes it from
+// the epilogue entirely).
+__global__ void fold_gain_kernel(const __nv_bfloat16* __restrict__ W2, const __nv_bfloat16* __restrict__ g,
+                                 __nv_bfloat16* __restrict__ W2g, int d, long long n_vec8) {
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  for (long long v = (long long)blockIdx.x * blockDim.x + threadIdx.x; v < n_vec8; v += stride) {
+    const long long e = v * 8;
+    const int j = (int)(e % d);
+    float w[8], gg[8];
+    unpack8(ldg_nc_v4(W2 + e), w);
+    unpack8(ldg_nc_v4(g + j), gg);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w[i] *= gg[i];
+    stg_v4(W2g + e, pack8(w));
+  }
+}
+
+// r_i = 1 / sqrt(sum_t P[i, t] / d + eps): the "very light auxiliary
+// reduction" that turns GEMM1's partial RMS into the RMSNorm row scale
+// (kucoin.com (ru) CODA article, «В «Финале» спрятаны сокровища»).
+__global__ void rms_rowreduce_kernel(const float* __restrict__ P, int T, float* __restrict__ r, int M,
+                                     float inv_d, float eps) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= M) return;
+  const float* row = P + (size_t)i * T;
+  float s = 0.f;
+  for (int t = 0; t < T; ++t) s += row[t];
+  r[i] = rsqrtf(fmaf(s, inv_d, eps));
+}
+
+template <int THREADS>
+__device__ __forceinline__ float block_sum(float v, float* scratch) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int w = threadIdx.x / 32;
+  if ((threadIdx.x & 31) == 0) scratch[w] = v;
+  __syncthreads();
+  float t = 0.f;
+  if (threadIdx.x < 32) {
+    t = threadIdx.x < THREADS / 32 ? scratch[threadIdx.x] : 0.f;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+  }
+  return t;  // valid in thread 0
+}
+
+// SwiGLU backward fused with the RMSNorm backward's row statistic, one block
+// per token row (F % 8 == 0):
+//   sigma = sigmoid(a); da = dY b sigma (1 + a (1 - sigma)); db = dY a sigma
+//   dA'  = bf16(r_i [da | db])            (the dn and dW2 GEMMs' left operand)
+//   c_i  = (r_i^2 / d) * sum_c (da a + db b)
+// c_i is the coefficient of the -c_i H_ij term of dH: with A = [a | b] the
+// pre-activations, sum_c dA_ic A_ic equals r_i sum_k dn_ik H_ik, so the whole
+// RMSNorm correction is a block-local epilogue term of the dn GEMM.
+constexpr int ROWSTAT_THREADS = 256;
+__global__ void __launch_bounds__(ROWSTAT_THREADS)
+    swiglu_bwd_rowstat_kernel(const __nv_bfloat16* __restrict__ dY, const __nv_bfloat16* __restrict__ AB,
+                              const float* __restrict__ r, __nv_bfloat16* __restrict__ dAp,
+                              float* __restrict__ c, int F, float inv_d) {
+  __shared__ float scratch[32];
+  const int row = blockIdx.x;
+  const __nv_bfloat16* dy = dY + (size_t)row * F;
+  const __nv_bfloat16* a = AB + (size_t)row * 2 * F;
+  const __nv_bfloat16* b = a + F;
+  __nv_bfloat16* oa = dAp + (size_t)row * 2 * F;
+  __nv_bfloat16* ob = oa + F;
+  const float rr = r[row];
+  float acc = 0.f;
+  for (int v = threadIdx.x; v < F / 8; v += ROWSTAT_THREADS) {
+    float fy[8], fa[8], fb[8], da[8], db[8];
+    unpack8(ldg_nc_v4(dy + 8 * v), fy);
+    unpack8(ldg_nc_v4(a + 8 * v), fa);
+    unpack8(ldg_nc_v4(b + 8 * v), fb);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float s = __frcp_rn(1.0f + __expf(-fa[i]));
+      da[i] = fy[i] * fb[i] * s * (1.f + fa[i] * (1.f - s));
+      db[i] = fy[i] * fa[i] * s;
+      acc = fmaf(da[i], fa[i], acc);
+      acc = fmaf(db[i], fb[i], acc);
+      da[i] *= rr;
+      db[i] *= rr;
+    }
+    stg_v4(oa + 8 * v, pack8(da));
+    stg_v4(ob + 8 * v, pack8(db));
+  }
+  const float tot = block_sum<ROWSTAT_THREADS>(acc, scratch);
+  if (threadIdx.x == 0) c[row] = rr * rr * inv_d * tot;
+}
+
+// dg_j = sum_t Pg[t, j]: reduce the dn GEMM's per-32-row column partials.
+__global__ void col_reduce_kernel(const float* __restrict__ Pg, int rows, int d, float* __restrict__ dg) {
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= d) return;
+  float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+  int t = 0;
+  for (; t + 4 <= rows; t += 4) {
+    s0 += Pg[(size_t)t * d + j];
+    s1 += Pg[(size_t)(t + 1) * d + j];
+    s2 += Pg[(size_t)(t + 2) * d + j];
+    s3 += Pg[(size_t)(t + 3) * d + j];
+  }
+  for (; t < rows; ++t) s0 += Pg[(size_t)t * d + j];
+  dg[j] = (s0 + s1) + (s2 + s3);
+}
+
+}  // namespace coda

@@ -1,0 +1,430 @@
+// Persistent, warp-specialised tcgen05 GEMM with fused epilogues (sm_100a).
+//
+// GEMM-epilogue structure (toolin.ai CODA article, section 核心の洞察; kucoin.com
+// (ru) CODA article, section «В «Финале» спрятаны сокровища»): a fixed mainloop
+// computes a 128 x 256 fp32 tile into tensor memory, and an epilogue transforms
+// the tile while it is still on chip before anything reaches HBM.  The
+// epilogue variants are built from the pages' primitives (five-primitive
+// table): elementwise transforms (residual add, SwiGLU, its backward),
+// vector loads (r, c, g), matrix-tile loads/stores (R, H, a/b, outputs) and
+// tile-wise reductions (row sums of squares, column sums for dg).
+//
+// Roles (192 threads, one CTA per SM):
+//   warp 0      TMA producer (one lane): 128B-swizzled K-major or MN-major
+//               operand tiles into a STAGES-deep shared-memory ring.
+//   warp 1      TMEM owner and MMA issuer (one lane): tcgen05.mma kind::f16,
+//               M=128 N=256 K=16, into one of two TMEM accumulators
+//               (2 x 256 columns), commit -> mbarriers.
+//   warps 2-5   epilogue: tcgen05.ld 32 lanes x 32 columns per step, one
+//               output row per thread, 16-byte global stores.
+// The two TMEM accumulators let tile i's epilogue overlap tile i+1's mainloop.
+#pragma once
+
+#include "coda_ptx.cuh"
+
+namespace coda {
+
+constexpr int BM = 128;              // tile rows (TMEM lanes)
+constexpr int BN = 256;              // tile columns (TMEM columns per accumulator)
+constexpr int BK = 64;               // reduction depth per stage (128 bytes of bf16)
+constexpr int STAGES = 4;
+constexpr int UMMA_K = 16;
+constexpr int A_STAGE_BYTES = BM * BK * 2;  // 16 KiB
+constexpr int B_STAGE_BYTES = BN * BK * 2;  // 32 KiB
+constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
+constexpr int MN_CHUNK_BYTES = 64 * BK * 2;  // one [64 k][64 mn] MN-major chunk, 8 KiB
+constexpr int NUM_THREADS = 192;
+constexpr uint32_t TMEM_COLS = 2 * BN;
+constexpr int GEMM_SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int GROUP_M = 16;          // tile rasterisation: 16 row tiles per group
+
+enum Epi : int {
+  EPI_STORE = 0,       // out = bf16(acc [* g_col])
+  EPI_RESID_RMS = 1,   // H = bf16(acc + R); P[row, ntile] = sum bf16(H)^2
+  EPI_SWIGLU = 2,      // a = r*acc_gate, b = r*acc_up; Y = silu(a)*b; AB = [a|b]
+  EPI_DN = 3,          // dH = g*acc - c*H (+dH_in); column partials of acc*H
+  EPI_SWIGLU_BWD = 4,  // dY = acc; da, db from a, b; dA = [da|db]
+};
+
+struct GemmParams {
+  int M;            // output rows
+  int N;            // output columns (EPI_SWIGLU / EPI_SWIGLU_BWD: F)
+  int K;            // reduction length
+  int num_m_tiles;
+  int num_n_tiles;
+  int k_blocks;
+  int split;        // EPI_SWIGLU: row offset of the up half in B and column offset of b in AB;
+                    // EPI_SWIGLU_BWD: column offset of b / db (= F)
+  __nv_bfloat16* out;
+  int ldo;
+  const __nv_bfloat16* in0;  // R (RESID_RMS), H (DN), AB (SWIGLU_BWD)
+  int ld_in0;
+  const __nv_bfloat16* in1;  // dH_in (DN), optional
+  const __nv_bfloat16* colvec;  // g (STORE scale, DN), optional for STORE
+  const float* rowvec;          // r (SWIGLU, optional), c (DN)
+  float* part;                  // P (RESID_RMS), Pg (DN)
+  int ld_part;
+  __nv_bfloat16* out2;          // AB (SWIGLU), optional
+  int ldo2;
+  uint32_t* status;
+  unsigned long long wait_limit_ns;
+  uint32_t kernel_id;
+};
+
+__device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int& m_blk, int& n_blk) {
+  const int group_size = GROUP_M * num_n;
+  const int group = tile / group_size;
+  const int first_m = group * GROUP_M;
+  const int gm = min(num_m - first_m, GROUP_M);
+  const int local = tile - group * group_size;
+  m_blk = first_m + local % gm;
+  n_blk = local / gm;
+}
+
+// Load 32 bf16 starting at p (16-byte aligned) as floats; zeros when !valid.
+__device__ __forceinline__ void load32_bf16(const __nv_bfloat16* p, bool valid, float (&f)[32]) {
+  if (valid) {
+    uint4 q[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) q[j] = ldg_nc_v4(p + 8 * j);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) unpack8(q[j], f + 8 * j);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) f[i] = 0.f;
+  }
+}
+
+__device__ __forceinline__ void store32_bf16(__nv_bfloat16* p, const float (&f)[32]) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) stg_v4(p + 8 * j, pack8(f + 8 * j));
+}
+
+// Sum of a 32 x 32 block held one row per lane, reduced over the lanes:
+// afterwards v[0] of lane l holds the sum over all lanes of column l.
+// Recursive halving: 16 + 8 + 4 + 2 + 1 shuffles for 32 columns.
+__device__ __forceinline__ void warp_column_sums(float (&v)[32], int lane) {
+#pragma unroll
+  for (int s = 16; s >= 1; s >>= 1) {
+    const bool upper = (lane & s) != 0;
+#pragma unroll
+    for (int i = 0; i < s; ++i) {
+      const float send = upper ? v[i] : v[i + s];
+      const float keep = upper ? v[i + s] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, s);
+    }
+  }
+}
+
+__device__ __forceinline__ float sigmoid_f(float x) { return __frcp_rn(1.0f + __expf(-x)); }
+
+template <int EPI>
+__device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbase, int row, bool rv, int m_blk,
+                                              int n_blk, int q, int lane) {
+  if constexpr (EPI == EPI_STORE) {
+    const int n0 = n_blk * BN;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      if (n0 + c >= p.N) break;
+      float v[32];
+      tmem_ld32(tbase + c, v);
+      if (p.colvec != nullptr) {
+        float g[32];
+        load32_bf16(p.colvec + n0 + c, true, g);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] *= g[i];
+      }
+      if (rv) store32_bf16(p.out + (size_t)row * p.ldo + n0 + c, v);
+    }
+  } else if constexpr (EPI == EPI_RESID_RMS) {
+    const int n0 = n_blk * BN;
+    float ss = 0.f;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      if (n0 + c >= p.N) break;
+      float rres[32];
+      load32_bf16(p.in0 + (size_t)row * p.ld_in0 + n0 + c, rv, rres);
+      float v[32];
+      tmem_ld32(tbase + c, v);
+      uint4 hq[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float h[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) h[i] = v[8 * j + i] + rres[8 * j + i];
+        hq[j] = pack8(h);
+        float hb[8];
+        unpack8(hq[j], hb);  // square the stored (bf16-rounded) H
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ss = fmaf(hb[i], hb[i], ss);
+      }
+      if (rv) {
+        __nv_bfloat16* dst = p.out + (size_t)row * p.ldo + n0 + c;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) stg_v4(dst + 8 * j, hq[j]);
+      }
+    }
+    if (rv) p.part[(size_t)row * p.ld_part + n_blk] = ss;
+  } else if constexpr (EPI == EPI_SWIGLU) {
+    constexpr int HALF = BN / 2;
+    const int n0 = n_blk * HALF;
+    const float rr = (p.rowvec != nullptr) ? (rv ? p.rowvec[row] : 0.f) : 1.f;
+#pragma unroll 1
+    for (int c = 0; c < HALF; c += 32) {
+      if (n0 + c >= p.N) break;
+      float a[32], b[32];
+      tmem_ld32(tbase + c, a);
+      tmem_ld32(tbase + HALF + c, b);
+      float y[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        a[i] *= rr;
+        b[i] *= rr;
+        y[i] = a[i] * sigmoid_f(a[i]) * b[i];
+      }
+      if (rv) {
+        store32_bf16(p.out + (size_t)row * p.ldo + n0 + c, y);
+        if (p.out2 != nullptr) {
+          store32_bf16(p.out2 + (size_t)row * p.ldo2 + n0 + c, a);
+          store32_bf16(p.out2 + (size_t)row * p.ldo2 + p.split + n0 + c, b);
+        }
+      }
+    }
+  } else if constexpr (EPI == EPI_DN) {
+    const int n0 = n_blk * BN;
+    const float cc = rv ? p.rowvec[row] : 0.f;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      if (n0 + c >= p.N) break;
+      float h[32];
+      load32_bf16(p.in0 + (size_t)row * p.ld_in0 + n0 + c, rv, h);
+      float v[32];
+      tmem_ld32(tbase + c, v);
+      float g[32];
+      load32_bf16(p.colvec + n0 + c, true, g);
+      float o[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) o[i] = fmaf(g[i], v[i], -cc * h[i]);
+      if (p.in1 != nullptr) {
+        float e[32];
+        load32_bf16(p.in1 + (size_t)row * p.ldo + n0 + c, rv, e);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] += e[i];
+      }
+      if (rv) store32_bf16(p.out + (size_t)row * p.ldo + n0 + c, o);
+      // dg partial: sum over this warp's 32 rows of acc * H, per column.
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] *= h[i];
+      warp_column_sums(v, lane);
+      p.part[(size_t)(m_blk * 4 + q) * p.ld_part + n0 + c + lane] = v[0];
+    }
+  } else if constexpr (EPI == EPI_SWIGLU_BWD) {
+    const int n0 = n_blk * BN;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      if (n0 + c >= p.N) break;
+      float a[32], b[32];
+      const __nv_bfloat16* ab = p.in0 + (size_t)row * p.ld_in0 + n0 + c;
+      load32_bf16(ab, rv, a);
+      load32_bf16(ab + p.split, rv, b);
+      float dy[32];
+      tmem_ld32(tbase + c, dy);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float s = sigmoid_f(a[i]);
+        const float da = dy[i] * b[i] * s * (1.f + a[i] * (1.f - s));
+        const float db = dy[i] * a[i] * s;
+        a[i] = da;
+        b[i] = db;
+      }
+      if (rv) {
+        __nv_bfloat16* dst = p.out + (size_t)row * p.ldo + n0 + c;
+        store32_bf16(dst, a);
+        store32_bf16(dst + p.split, b);
+      }
+    }
+  }
+}
+
+template <int EPI, bool A_MN, bool B_MN>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * A_STAGE_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * B_STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* mma_done = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const WaitCtl ctl{abort_flag, p.status, p.wait_limit_ns, p.kernel_id};
+  const int num_tiles = p.num_m_tiles * p.num_n_tiles;
+  int issued = 0;  // TMA stages issued by the producer lane
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------------------- producer
+      const uint64_t hint = l2_policy_evict_normal();
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        int m_blk, n_blk;
+        tile_coords(tile, p.num_m_tiles, p.num_n_tiles, m_blk, n_blk);
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, ctl, 0, kWaitEmpty)) {
+            ok = false;
+            break;
+          }
+          uint64_t* bar = &full[stage];
+          mbar_arrive_expect_tx(bar, STAGE_BYTES);
+          uint8_t* a_dst = sA + stage * A_STAGE_BYTES;
+          uint8_t* b_dst = sB + stage * B_STAGE_BYTES;
+          const int k0 = kb * BK;
+          if constexpr (!A_MN) {
+            tma_load_2d(a_dst, &tmA, bar, k0, m_blk * BM, hint);
+          } else {
+#pragma unroll
+            for (int c = 0; c < BM / 64; ++c) tma_load_2d(a_dst + c * MN_CHUNK_BYTES, &tmA, bar, m_blk * BM + c * 64, k0, hint);
+          }
+          if constexpr (EPI == EPI_SWIGLU) {
+            tma_load_2d(b_dst, &tmB, bar, k0, n_blk * (BN / 2), hint);
+            tma_load_2d(b_dst + B_STAGE_BYTES / 2, &tmB, bar, k0, p.split + n_blk * (BN / 2), hint);
+          } else if constexpr (!B_MN) {
+            tma_load_2d(b_dst, &tmB, bar, k0, n_blk * BN, hint);
+          } else {
+#pragma unroll
+            for (int c = 0; c < BN / 64; ++c) tma_load_2d(b_dst + c * MN_CHUNK_BYTES, &tmB, bar, n_blk * BN + c * 64, k0, hint);
+          }
+          ++issued;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------------------------------------------------------- MMA issuer
+      constexpr uint32_t idesc = make_idesc_bf16(BM, BN, A_MN, B_MN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, ctl, 1, kWaitAccEmpty)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          if (!mbar_wait(&full[stage], phase, ctl, 1, kWaitFull)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(sA + stage * A_STAGE_BYTES);
+          const uint32_t b_base = smem_u32(sB + stage * B_STAGE_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / UMMA_K; ++k) {
+            // K-major: advance 16 elements (32 B) inside the 128-B swizzled row;
+            // MN-major: advance 16 k-rows of 128 B (2 KiB), chunks of 64 mn 8 KiB apart.
+            const uint64_t ad = A_MN ? make_sdesc_sw128(a_base + k * 2048, MN_CHUNK_BYTES, 1024)
+                                     : make_sdesc_sw128(a_base + k * 32, 16, 1024);
+            const uint64_t bd = B_MN ? make_sdesc_sw128(b_base + k * 2048, MN_CHUNK_BYTES, 1024)
+                                     : make_sdesc_sw128(b_base + k * 32, 16, 1024);
+            umma_bf16(d_tmem, ad, bd, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+          }
+          umma_commit(&empty[stage]);  // frees the stage once these MMAs have read it
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);  // accumulator ready for the epilogue
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      // Every MMA issued by this thread has completed once mma_done fires.
+      umma_commit(mma_done);
+      mbar_wait(mma_done, 0, ctl, 1, kWaitDrain);
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      int m_blk, n_blk;
+      tile_coords(tile, p.num_m_tiles, p.num_n_tiles, m_blk, n_blk);
+      // Warp-uniform outcome: tcgen05.ld below needs all 32 lanes converged.
+      const bool ok = mbar_wait(&tfull[acc], acc_phase, ctl, 2 + q, kWaitAccFull);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
+      const int row = m_blk * BM + q * 32 + lane;
+      epilogue_tile<EPI>(p, tbase, row, row < p.M, m_blk, n_blk, q, lane);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag) {
+    // A role gave up: let the last (up to STAGES) copies land before the
+    // CTA's shared memory is released.  Every wait here is bounded too.
+    if (warp == 0 && lane == 0) {
+      const int first = issued > STAGES ? issued - STAGES : 0;
+      for (int i = first; i < issued; ++i) {
+        const uint32_t par = (uint32_t)((i / STAGES) & 1);
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(&full[i % STAGES], par) && global_timer_ns() - t0 < ctl.limit_ns) {
+        }
+      }
+    }
+    __syncthreads();
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+}  // namespace coda

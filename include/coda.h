@@ -1,0 +1,204 @@
+/*
+ * coda.h — C ABI of the B200 (sm_100a) GEMM-epilogue library for the CODA
+ * GEMM-Residual-RMSNorm-GEMM(+SwiGLU) block and the SwiGLU MLP.
+ *
+ * The method (toolin.ai, "CODA：LLMと初心者が光速のGPUカーネルを書けるようにする",
+ * section 核心の洞察; kucoin.com (ru) "CODA: ...", section
+ * «В «Финале» спрятаны сокровища»): memory-bound Transformer operations are
+ * rewritten so they run in the epilogue of a GEMM while the GEMM's output is
+ * still on chip.  In GEMM -> RMSNorm -> GEMM the RMSNorm row scale r commutes
+ * with the second GEMM, so GEMM1's epilogue only adds the residual and emits
+ * per-tile partial sums of squares, a light reduction turns them into r, and
+ * GEMM2's epilogue applies r (and here SwiGLU).  The same structure carries to
+ * the backward pass (kucoin (ru), same section: a block-local forward epilogue
+ * gives a backward of the same form) and to SwiGLU.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *    never allocates, frees or synchronises in these calls; all work is
+ *    enqueued on `stream` (a cudaStream_t passed as void*, NULL = legacy
+ *    default stream) and runs asynchronously.
+ *  - "bf16" arrays hold IEEE bfloat16 values (uint16 bit patterns), row-major,
+ *    densely packed (leading dimension = number of columns).  fp32 arrays are
+ *    IEEE float, also densely packed.
+ *  - Weights use the [out_features, in_features] layout, so the pages'
+ *    "X * W1" is X[M,K] times W1[d,K]^T.
+ *  - Gate/up weights stack the F gate rows first and the F up rows after them
+ *    ([2F, d]); saved pre-activations AB[M, 2F] hold a in columns [0, F) and
+ *    b in columns [F, 2F).
+ *  - Alignment: every pointer must be 16-byte aligned.  Shape requirements are
+ *    stated per call; violations return an error code and launch nothing.
+ *  - `ws` is a caller-owned device workspace of at least the size returned by
+ *    the matching *_workspace_bytes() query.  Its first 256 bytes hold a
+ *    device status word: kernels record bounded-wait timeouts there.  Zero it
+ *    once (coda_status_clear) before first use; it is sticky until cleared.
+ *  - The return value reports host-detectable errors only (arguments, shapes,
+ *    alignment, device capability, launch failures).  Device-side errors are
+ *    read with coda_status_query().  No call aborts or throws.
+ *  - Requires an sm_100 device (B200); otherwise CODA_ERR_NO_SM100.
+ */
+#ifndef CODA_H_
+#define CODA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  CODA_OK = 0,
+  CODA_ERR_INVALID_ARG = 1,         /* null pointer, non-positive size, eps <= 0 */
+  CODA_ERR_UNSUPPORTED_SHAPE = 2,   /* a dimension violates the stated multiple */
+  CODA_ERR_MISALIGNED = 3,          /* a pointer is not 16-byte aligned */
+  CODA_ERR_WORKSPACE_TOO_SMALL = 4, /* ws_bytes below the *_workspace_bytes() size */
+  CODA_ERR_NO_SM100 = 5,            /* current device is not compute capability 10.x */
+  CODA_ERR_CUDA = 6,                /* a CUDA runtime call or kernel launch failed */
+  CODA_ERR_DEVICE_TIMEOUT = 7       /* (status word) a device-side wait gave up */
+} coda_status;
+
+/* Static human-readable name of a status code. */
+const char* coda_status_string(int status);
+
+/* Library version as an integer (major*10000 + minor*100 + patch). */
+int coda_version(void);
+
+/* ---------------------------------------------------------------- status word */
+
+/* Enqueue a zeroing of the workspace's status word on `stream`. */
+coda_status coda_status_clear(void* ws, void* stream);
+
+/* Synchronise `stream`, then read the workspace's status word.  Returns
+ * CODA_OK, or the device-side error recorded by a kernel (for a timeout,
+ * CODA_ERR_DEVICE_TIMEOUT).  If `detail` is non-null it receives the raw
+ * 32-bit detail word (kernel id << 16 | role << 8 | reason). */
+coda_status coda_status_query(const void* ws, void* stream, uint32_t* detail);
+
+/* Set the per-wait limit of device-side bounded waits, in nanoseconds, for
+ * launches issued after this call from any host thread (default 4e9 = 4 s).
+ * Values are clamped to [1e3, 6e10]. */
+void coda_set_wait_limit_ns(uint64_t ns);
+
+/* ---------------------------------------------------------------- building block */
+
+/* C[M,N] (bf16) = op(A) * op(B)^T with fp32 accumulation on tcgen05 tensor cores.
+ *   a_mn_major = 0: A stored [M, K] (K contiguous);  1: A stored [K, M].
+ *   b_mn_major = 0: B stored [N, K];                1: B stored [K, N].
+ * Requires M, N >= 1, K >= 1; N % 32 == 0; the contiguous dimension of every
+ * operand a multiple of 8 (16-byte rows).  Rows/columns beyond the extents are
+ * zero-filled on load and masked on store.  ws: coda_gemm_workspace_bytes(). */
+size_t coda_gemm_workspace_bytes(void);
+coda_status coda_gemm(const void* A, const void* B, void* C, int M, int N, int K,
+                      int a_mn_major, int b_mn_major, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------- gain fold */
+
+/* W2g[n, j] = bf16(g[j] * W2[n, j]) for the [N, d] gate/up weight: the RMSNorm
+ * gain folded into the second GEMM's weight, diag(g) * W2 in the pages'
+ * column-vector notation.  Requires d % 8 == 0. */
+coda_status coda_fold_gain(const void* W2, const void* g, void* W2g, int d, int N, void* stream);
+
+/* ---------------------------------------------------------------- GEMM + SwiGLU epilogue */
+
+/* The gate/up GEMM-epilogue program on its own (toolin.ai §核心の洞察: r applied
+ * in the second GEMM's epilogue; five-primitive table: activation as an
+ * elementwise transform, a/b saved by the matrix-tile store):
+ *   acc = A Wgu^T (fp32);  a = s_i acc[:, :F], b = s_i acc[:, F:] with
+ *   s_i = r[i] (or 1 when r_or_null is null);  Y = silu(a) * b;  AB = [a | b].
+ * Inputs A [M,K] bf16, Wgu [2F,K] bf16 (gate rows first), r_or_null [M] fp32.
+ * Outputs Y [M,F] bf16, AB_or_null [M,2F] bf16.  Requires K % 64 == 0,
+ * F % 64 == 0.  ws: coda_gemm_workspace_bytes(). */
+coda_status coda_gemm_swiglu(const void* A, const void* Wgu, const float* r_or_null, void* Y, void* AB_or_null,
+                             int M, int K, int F, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------- GRG forward */
+
+/* Workspace for coda_grg_fwd: status word, per-tile partial sums of squares
+ * P[M, d/256] fp32, and (when the caller passes no pre-folded weight) W2g. */
+size_t coda_grg_fwd_workspace_bytes(int M, int K, int d, int N, int prefolded);
+
+/* Forward of GEMM -> residual -> partial RMS -> GEMM -> SwiGLU
+ * (toolin.ai §核心の洞察; kucoin (ru) §«В «Финале» спрятаны сокровища»):
+ *   GEMM1 epilogue:  H = X W1^T + R (fp32 accumulate + fp32(R), stored bf16),
+ *                    P[i, t] = sum_{j in tile t} bf16(H_ij)^2 (tiles of 256 columns)
+ *   row reduce:      r_i = 1 / sqrt(sum_t P[i,t] / d + eps)            (fp32 [M])
+ *   GEMM2 epilogue:  acc = H W2g^T with W2g = W2 diag(g);  a = r_i acc_gate,
+ *                    b = r_i acc_up;  Y = silu(a) * b  (bf16 [M, F]);
+ *                    AB = [a | b] (bf16 [M, 2F]) saved for the backward.
+ * Inputs:  X [M,K], W1 [d,K], R [M,d], g [d], W2 [N=2F, d] (all bf16).
+ *          W2g_or_null: optional caller-folded diag(g)-scaled W2 [N, d]; when
+ *          null the fold runs inside this call into the workspace.
+ * Outputs: H [M,d] bf16, r [M] fp32, Y [M,F] bf16, AB_or_null [M,N] bf16.
+ * Requires M >= 1, K % 64 == 0, d % 64 == 0, N % 128 == 0 (F % 64 == 0), eps > 0.
+ * Rows, the last partial-RMS tile and the last F tile may be ragged. */
+coda_status coda_grg_fwd(const void* X, const void* W1, const void* R, const void* g,
+                         const void* W2, const void* W2g_or_null,
+                         void* H, float* r, void* Y, void* AB_or_null,
+                         int M, int K, int d, int N, float eps,
+                         void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------- GRG backward */
+
+/* Workspace for coda_grg_bwd: status word, dA' [M, N] bf16, c [M] fp32 and
+ * column partials Pg [ceil(M/32), d] fp32. */
+size_t coda_grg_bwd_workspace_bytes(int M, int K, int d, int N);
+
+/* Backward of the block for the loss <dY, Y> + <dH_in, H> (toolin.ai §実験結果,
+ * GEMM-Residual-PartialRMS-GEMM backward).  Steps, each a GEMM + epilogue or a
+ * light pass:
+ *   SwiGLU bwd + row stat:  da, db from dY, a, b;  dA' = bf16(r_i [da | db]);
+ *                           c_i = (r_i^2 / d) sum_c dA_ic A_ic
+ *   dn GEMM + epilogue:     dR = dH = g_j (dA' W2)_ij - c_i H_ij (+ dH_in)
+ *                           with column partials of (dA' W2)_ij H_ij for dg
+ *   column reduce:          dg_j = sum_i (dA' W2)_ij H_ij
+ *   dW2 GEMM + epilogue:    dW2 = g_j (dA'^T H)_cj
+ *   plain GEMMs:            dX = dH W1,  dW1 = dH^T X
+ * Inputs:  dY [M,F], dH_in_or_null [M,d], X [M,K], W1 [d,K], H [M,d] and
+ *          r [M] fp32 and AB [M,N] from coda_grg_fwd, g [d], W2 [N,d].
+ * Outputs: dX [M,K], dR [M,d] (= dH), dW1 [d,K], dW2 [N,d] (bf16), dg [d] fp32.
+ * Requires the same shape rules as coda_grg_fwd. */
+coda_status coda_grg_bwd(const void* dY, const void* dH_in_or_null,
+                         const void* X, const void* W1, const void* H, const float* r,
+                         const void* AB, const void* g, const void* W2,
+                         void* dX, void* dR, void* dW1, void* dW2, float* dg,
+                         int M, int K, int d, int N,
+                         void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------- SwiGLU MLP */
+
+/* Workspace for coda_swiglu_fwd (status word only). */
+size_t coda_swiglu_fwd_workspace_bytes(int M, int d, int F);
+
+/* SwiGLU MLP forward (toolin.ai five-primitive table: activation as an
+ * elementwise epilogue transform):
+ *   gate/up GEMM + epilogue: A = X Wgu^T;  Y = silu(a) * b;  AB = [a | b]
+ *   down GEMM:               Out = Y Wdown^T
+ * Inputs X [M,d], Wgu [2F,d], Wdown [d,F].  Outputs Y [M,F], AB_or_null
+ * [M,2F], Out [M,d] (bf16).  Requires M >= 1, d % 64 == 0, F % 64 == 0. */
+coda_status coda_swiglu_fwd(const void* X, const void* Wgu, const void* Wdown,
+                            void* Y, void* AB_or_null, void* Out,
+                            int M, int d, int F, void* ws, size_t ws_bytes, void* stream);
+
+/* Workspace for coda_swiglu_bwd: status word and dA [M, 2F] bf16. */
+size_t coda_swiglu_bwd_workspace_bytes(int M, int d, int F);
+
+/* SwiGLU MLP backward for the loss <dOut, Out> (toolin.ai §実験結果, SwiGLU backward):
+ *   down dgrad GEMM + SwiGLU-bwd epilogue:  dY = dOut Wdown, then
+ *       da = dY b sigmoid(a) (1 + a (1 - sigmoid(a))), db = dY silu(a);
+ *       dA = [da | db] (bf16, workspace)
+ *   plain GEMMs:  dWdown = dOut^T Y,  dWgu = dA^T X,  dX = dA Wgu
+ * Inputs dOut [M,d], X [M,d], Wgu [2F,d], Wdown [d,F], Y [M,F], AB [M,2F].
+ * Outputs dX [M,d], dWgu [2F,d], dWdown [d,F] (bf16).  Same shape rules as
+ * coda_swiglu_fwd. */
+coda_status coda_swiglu_bwd(const void* dOut, const void* X, const void* Wgu, const void* Wdown,
+                            const void* Y, const void* AB,
+                            void* dX, void* dWgu, void* dWdown,
+                            int M, int d, int F, void* ws, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CODA_H_ */

@@ -1,0 +1,202 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 CPU oracle.
+
+Small and ragged shapes that span several tiles and a ragged tail, compared
+element by element with |gpu - ref| <= 1e-2 |ref| + 1e-2 rms(ref) for bf16
+outputs and 1e-3 relative for r against the oracle at the method's storage
+precision (the *_stored functions: the same fp64 arithmetic with each tensor
+the method stores between passes rounded to bf16), and against the pure fp64
+oracle within the bound derived from that storage rounding (tests/parity.py);
+plus structured cases whose integer tile/row indexing is checked bit-exactly.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from gemm_epilogue_fusion_tmem_b200 import synth
+from oracle import coda_oracle as O
+from tests.parity import BWD_OUTLIER_FRAC, assert_pure, assert_rel, assert_tol, f64
+
+pytestmark = pytest.mark.gpu
+
+
+def _cuda(d):
+    return {k: v.cuda() for k, v in d.items()}
+
+
+# ----------------------------------------------------------------------------- plain GEMM core
+
+GEMM_CASES = [
+    # (M, N, K): ragged M, ragged N tile, several k-blocks
+    (200, 512, 320),
+    (1, 256, 64),
+    (384, 288, 4160),
+    (2048, 4096, 256),  # 256 tiles > 148 SMs: persistent loop, both TMEM accumulators
+]
+
+
+@pytest.mark.parametrize("a_mn", [False, True])
+@pytest.mark.parametrize("b_mn", [False, True])
+@pytest.mark.parametrize("M,N,K", GEMM_CASES)
+def test_gemm_core(cuda_lib, M, N, K, a_mn, b_mn):
+    if a_mn and M % 8:
+        pytest.skip("MN-major A needs M % 8 == 0")
+    t = synth.gemm_inputs(M, N, K, seed=M + N + K)
+    A, B = t["A"], t["B"]
+    Ad = A.t().contiguous().cuda() if a_mn else A.cuda()
+    Bd = B.t().contiguous().cuda() if b_mn else B.cuda()
+    C = cuda_lib.gemm(Ad, Bd, M, N, K, a_mn_major=a_mn, b_mn_major=b_mn)
+    torch.cuda.synchronize()
+    assert_tol(C, O.gemm(f64(A), f64(B)), f"gemm M={M} N={N} K={K} a_mn={a_mn} b_mn={b_mn}")
+
+
+def test_gemm_ragged_reduction_mn_major(cuda_lib):
+    """Reduction length not a multiple of the 64-deep stage (zero-filled tail), both MN-major."""
+    M, N, K = 256, 512, 200
+    t = synth.gemm_inputs(M, N, K, seed=3)
+    C = cuda_lib.gemm(t["A"].t().contiguous().cuda(), t["B"].t().contiguous().cuda(), M, N, K, True, True)
+    torch.cuda.synchronize()
+    assert_tol(C, O.gemm(f64(t["A"]), f64(t["B"])), "gemm ragged K")
+
+
+# ----------------------------------------------------------------------------- GRG forward / backward
+
+GRG_CASES = [
+    # (M, K, d, F, eps)
+    (256, 512, 512, 1024, 1e-6),     # the tiny workload
+    (200, 320, 384, 320, 1e-5),      # ragged M, ragged partial-RMS tile, ragged F tile, K != d
+    (1, 64, 256, 128, 1e-6),         # a single token
+    (2048, 1024, 1024, 2816, 1e-6),  # > 148 tiles in the gate/up GEMM
+]
+
+
+def _grg_oracle(t, eps, with_dH_in=False):
+    X, W1, R, g, W2, dY = (f64(t[k]) for k in ("X", "W1", "R", "g", "W2", "dY"))
+    dH_in = f64(t["dH_in"]) if with_dH_in else None
+    fwd = O.grg_forward(X, W1, R, g, W2, eps)
+    bwd = O.grg_backward(dY, X, W1, R, g, W2, eps, dH_in=dH_in, fwd=fwd)
+    fwd_s = O.grg_forward_stored(X, W1, R, g, W2, eps)
+    bwd_s = O.grg_backward_stored(dY, X, W1, R, g, W2, eps, dH_in=dH_in, fwd=fwd_s)
+    return fwd, bwd, fwd_s, bwd_s
+
+
+def _check_fwd(o, fwd, fwd_s, tag):
+    F = fwd["a"].shape[1]
+    gpu = {"H": o["H"], "Y": o["Y"], "a": o["AB"][:, :F], "b": o["AB"][:, F:]}
+    for k, v in gpu.items():
+        assert_tol(v, fwd_s[k], f"{tag} {k}")
+        assert_pure(v, fwd[k], f"{tag} {k}")
+    assert_rel(o["r"], fwd_s["r"], f"{tag} r")
+    assert_rel(o["r"], fwd["r"], f"{tag} r (vs pure fp64)")
+
+
+@pytest.mark.parametrize("M,K,d,F,eps", GRG_CASES)
+def test_grg_forward(cuda_lib, M, K, d, F, eps):
+    t = synth.grg_inputs(M, K, d, F, seed=1)
+    td = _cuda(t)
+    o = cuda_lib.grg_fwd(td["X"], td["W1"], td["R"], td["g"], td["W2"], eps)
+    torch.cuda.synchronize()
+    fwd, _, fwd_s, _ = _grg_oracle(t, eps)
+    _check_fwd(o, fwd, fwd_s, f"grg_fwd M={M} K={K} d={d} F={F}")
+
+
+def test_grg_forward_prefolded_weight(cuda_lib):
+    M, K, d, F, eps = 256, 512, 512, 1024, 1e-6
+    t = synth.grg_inputs(M, K, d, F, seed=2)
+    td = _cuda(t)
+    W2g = cuda_lib.fold_gain(td["W2"], td["g"])
+    o = cuda_lib.grg_fwd(td["X"], td["W1"], td["R"], td["g"], td["W2"], eps, W2g=W2g)
+    torch.cuda.synchronize()
+    assert_tol(W2g, f64(t["W2"]) * f64(t["g"])[None, :], "W2g", rel=4e-3, rms_frac=0.0)
+    fwd, _, fwd_s, _ = _grg_oracle(t, eps)
+    _check_fwd(o, fwd, fwd_s, "grg_fwd prefolded")
+
+
+@pytest.mark.parametrize("with_dH_in", [False, True])
+@pytest.mark.parametrize("M,K,d,F,eps", GRG_CASES)
+def test_grg_backward(cuda_lib, M, K, d, F, eps, with_dH_in):
+    t = synth.grg_inputs(M, K, d, F, seed=4, dH_in=with_dH_in)
+    td = _cuda(t)
+    o = cuda_lib.grg_fwd(td["X"], td["W1"], td["R"], td["g"], td["W2"], eps)
+    b = cuda_lib.grg_bwd(td["dY"], td["X"], td["W1"], o["H"], o["r"], o["AB"], td["g"], td["W2"],
+                         dH_in=td.get("dH_in"))
+    torch.cuda.synchronize()
+    _, bwd, _, bwd_s = _grg_oracle(t, eps, with_dH_in)
+    tag = f"grg_bwd M={M} K={K} d={d} F={F} dH_in={with_dH_in}"
+    for k in ("dX", "dR", "dW1", "dW2", "dg"):
+        assert_tol(b[k], bwd_s[k], f"{tag} {k}", outlier_frac=BWD_OUTLIER_FRAC)
+        assert_pure(b[k], bwd[k], f"{tag} {k}")
+
+
+def test_grg_structured_exact_indexing(cuda_lib):
+    """X = 0, R one-hot v at (i, j), W2 = [I; I], g = 1 (F = d).
+
+    Then H = R exactly, the partial sum of squares is v^2 in cell (i, j // 256)
+    and 0 elsewhere (bit-exact tile/row indexing), r_i = 1/sqrt(v^2/d + eps),
+    every other row has r = 1/sqrt(eps), and a = b = r H.
+    """
+    M, K, d, eps, v = 300, 128, 768, 1e-6, 3.0
+    F = d
+    X = torch.zeros(M, K, dtype=torch.bfloat16)
+    W1 = synth.gemm_inputs(d, 32, K, seed=5)["A"]
+    eye = torch.eye(d, dtype=torch.bfloat16)
+    W2 = torch.cat([eye, eye], dim=0)
+    g = torch.ones(d, dtype=torch.bfloat16)
+    for (i, j) in [(0, 0), (131, 300), (299, 767), (257, 511)]:
+        R = torch.zeros(M, d, dtype=torch.bfloat16)
+        R[i, j] = v
+        ws = cuda_lib.Workspace(cuda_lib.library().coda_grg_fwd_workspace_bytes(M, K, d, 2 * F, 0))
+        o = cuda_lib.grg_fwd(X.cuda(), W1.cuda(), R.cuda(), g.cuda(), W2.cuda(), eps, ws=ws)
+        torch.cuda.synchronize()
+        assert torch.equal(o["H"].cpu(), R), "H must equal R bit for bit"
+        T = -(-d // 256)
+        P = ws.buf[256:256 + M * T * 4].view(torch.float32).view(M, T).cpu().numpy()
+        expect = np.zeros((M, T), dtype=np.float32)
+        expect[i, j // 256] = v * v
+        np.testing.assert_array_equal(P, expect)
+        r_exp = np.full(M, 1.0 / np.sqrt(eps))
+        r_exp[i] = 1.0 / np.sqrt(v * v / d + eps)
+        assert_rel(o["r"], r_exp, "r one-hot")
+        a = f64(o["AB"][:, :F])
+        b = f64(o["AB"][:, F:])
+        np.testing.assert_array_equal(a, b)
+        assert a[i, j] == pytest.approx(r_exp[i] * v, rel=1e-2)
+        a[i, j] = 0.0
+        assert not np.any(a), "only the one-hot entry may be nonzero"
+
+
+# ----------------------------------------------------------------------------- SwiGLU MLP
+
+SWIGLU_CASES = [
+    (200, 256, 320),
+    (512, 512, 1024),
+    (1, 64, 64),
+]
+
+
+@pytest.mark.parametrize("M,d,F", SWIGLU_CASES)
+def test_swiglu_forward_backward(cuda_lib, M, d, F):
+    t = synth.swiglu_inputs(M, d, F, seed=6)
+    td = _cuda(t)
+    o = cuda_lib.swiglu_fwd(td["X"], td["Wgu"], td["Wdown"])
+    b = cuda_lib.swiglu_bwd(td["dOut"], td["X"], td["Wgu"], td["Wdown"], o["Y"], o["AB"])
+    torch.cuda.synchronize()
+    X, Wgu, Wdown, dOut = (f64(t[k]) for k in ("X", "Wgu", "Wdown", "dOut"))
+    fwd = O.swiglu_forward(X, Wgu, Wdown)
+    bwd = O.swiglu_backward(dOut, X, Wgu, Wdown, fwd=fwd)
+    fwd_s = O.swiglu_forward_stored(X, Wgu, Wdown)
+    bwd_s = O.swiglu_backward_stored(dOut, X, Wgu, Wdown, fwd=fwd_s)
+    tag = f"swiglu M={M} d={d} F={F}"
+    gpu = {"Y": o["Y"], "a": o["AB"][:, :F], "b": o["AB"][:, F:], "Out": o["Out"],
+           "dX": b["dX"], "dWgu": b["dWgu"], "dWdown": b["dWdown"]}
+    for k, v in gpu.items():
+        ref_s = fwd_s[k] if k in fwd_s else bwd_s[k]
+        ref = fwd[k] if k in fwd else bwd[k]
+        assert_tol(v, ref_s, f"{tag} {k}")
+        assert_pure(v, ref, f"{tag} {k}")
+
+
+def test_status_word_stays_clear(cuda_lib):
+    ws = cuda_lib.workspace(1 << 20)
+    st, detail = ws.query()
+    assert st == 0 and detail == 0, f"device status {st} detail {detail:#x}"
