@@ -477,3 +477,69 @@ coda_status coda_swiglu_bwd(const void* dOut, const void* X, const void* Wgu, co
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------ forward without allocation
+//
+// For callers that cannot allocate device memory.  The scratch of the GRG
+// forward (status word + partial sums of squares) lives in this file-scope
+// device array instead of a caller workspace.  In host code the name
+// g_static_scratch is only a host-side stand-in: the device address comes
+// from cudaGetSymbolAddress, looked up once per device with that device
+// current and cached.  All calls on a device share the array.
+
+namespace coda {
+namespace {
+constexpr size_t kStaticScratchBytes = kStatusBytes + (size_t)CODA_STATIC_PARTIALS_MAX * sizeof(float);
+__device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+std::atomic<void*> g_static_scratch_addr[64];
+
+coda_status static_scratch(int dev, void** out) {
+  void* p = g_static_scratch_addr[dev].load();
+  if (p == nullptr) {
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) return CODA_ERR_CUDA;
+    g_static_scratch_addr[dev].store(p);
+  }
+  *out = p;
+  return CODA_OK;
+}
+}  // namespace
+}  // namespace coda
+
+extern "C" coda_status coda_grg_fwd_prefolded_static(const void* X, const void* W1, const void* R, const void* W2g,
+                                                     void* H, float* r, void* Y, void* AB_or_null, int M, int K,
+                                                     int d, int N, float eps, void* stream) {
+  if (!X || !W1 || !R || !W2g || !H || !r || !Y) return CODA_ERR_INVALID_ARG;
+  if (!(eps > 0.f)) return CODA_ERR_INVALID_ARG;
+  CODA_TRY(check_grg_shapes(M, K, d, N));
+  const void* ptrs[] = {X, W1, R, W2g, H, r, Y, AB_or_null};
+  for (const void* q : ptrs)
+    if (q && !aligned16(q)) return CODA_ERR_MISALIGNED;
+  const int T = cdiv(d, kRmsTile);
+  if ((unsigned long long)M * (unsigned long long)T > (unsigned long long)CODA_STATIC_PARTIALS_MAX)
+    return CODA_ERR_WORKSPACE_TOO_SMALL;  // the static scratch is too small for this shape
+  int dev;
+  CODA_TRY(current_device(dev));
+  void* scratch = nullptr;
+  CODA_TRY(static_scratch(dev, &scratch));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // The status word must start at zero; P is fully overwritten by GEMM1's epilogue.
+  CODA_TRY(launch_status(cudaMemsetAsync(scratch, 0, kStatusBytes, s)));
+  float* P = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + kStatusBytes);
+  const int F = N / 2;
+  {
+    CUtensorMap ta, tb;
+    if (!make_operand_map(&ta, X, M, K, false, BM) || !make_operand_map(&tb, W1, d, K, false, BN))
+      return CODA_ERR_CUDA;
+    GemmParams p = base_params(M, d, K, BN, scratch);
+    p.out = bf(H);
+    p.ldo = d;
+    p.in0 = cbf(R);
+    p.ld_in0 = d;
+    p.part = P;
+    p.ld_part = T;
+    CODA_TRY((launch_gemm<EPI_RESID_RMS, false, false>(ta, tb, p, s)));
+  }
+  rms_rowreduce_kernel<<<cdiv(M, 256), 256, 0, s>>>(P, T, r, M, 1.0f / (float)d, eps);
+  CODA_TRY(launch_status(cudaPeekAtLastError()));
+  return gemm_swiglu(H, W2g, r, Y, AB_or_null, M, d, F, scratch, s);
+}

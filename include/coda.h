@@ -197,6 +197,51 @@ coda_status coda_swiglu_bwd(const void* dOut, const void* X, const void* Wgu, co
                             void* dX, void* dWgu, void* dWdown,
                             int M, int d, int F, void* ws, size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------- forward without any allocation */
+
+/* Upper bound on M * ceil(d / 256) for coda_grg_fwd_prefolded_static: the
+ * partial sums of squares it keeps in the library's own static scratch
+ * (4 MiB of fp32, e.g. M = 32768 tokens at d = 8192). */
+#define CODA_STATIC_PARTIALS_MAX (1u << 20)
+
+/* The GRG forward for callers that cannot allocate device memory: code that
+ * runs where cudaMalloc is not allowed or not wanted (inside a framework that
+ * owns every device byte through its own arena, a plugin interface that
+ * hands over inputs and outputs but no workspace, a serving loop that must
+ * not allocate on the request path).  The pages describe no such entry point;
+ * it exists for those callers only.
+ *
+ * Computes exactly what coda_grg_fwd computes when given a pre-folded weight
+ * (same kernels, same results): GEMM1 + residual + partial sums of squares,
+ * the row reduce to r, GEMM2 + r + SwiGLU.  The caller passes every input and
+ * output (X [M,K], W1 [d,K], R [M,d], W2g = bf16(W2 diag(g)) [N,d] from
+ * coda_fold_gain, H [M,d], r [M] fp32, Y [M,F], AB_or_null [M,N]); there is no
+ * ws argument.  Its only scratch, the partial sums P[M, ceil(d/256)] and a
+ * device status word, lives in a file-scope __device__ array of the library
+ * (4 MiB + 256 bytes), which every GPU that loads the library keeps until the
+ * process exits.  No cudaMalloc, cudaFree or other allocating call is made.
+ *
+ * Limits and behaviour:
+ *  - M * ceil(d/256) above CODA_STATIC_PARTIALS_MAX returns
+ *    CODA_ERR_WORKSPACE_TOO_SMALL before anything is enqueued ("the static
+ *    scratch is too small for this shape"); the other shape rules are those of
+ *    coda_grg_fwd.
+ *  - The first call on a device (with that device current) looks up the
+ *    array's device address with cudaGetSymbolAddress and caches it; make
+ *    that first call before any stream capture.  A failed lookup returns
+ *    CODA_ERR_CUDA.
+ *  - Every call on a device shares the one array, and the array keeps the
+ *    last call's contents.  Each call zeroes the status word first (the
+ *    partial sums are fully overwritten); calls whose work overlaps on the GPU
+ *    (different streams, or host threads without ordering) race on the array,
+ *    so callers must serialise them.
+ *  - A device-side wait timeout is recorded in that internal status word,
+ *    which callers cannot read; use coda_grg_fwd with a workspace when the
+ *    device status must be observable. */
+coda_status coda_grg_fwd_prefolded_static(const void* X, const void* W1, const void* R, const void* W2g,
+                                          void* H, float* r, void* Y, void* AB_or_null,
+                                          int M, int K, int d, int N, float eps, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

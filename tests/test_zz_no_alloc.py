@@ -1,0 +1,63 @@
+"""The allocation-free GRG forward (coda_grg_fwd_prefolded_static) against coda_grg_fwd.
+
+Some callers cannot allocate device memory (a framework arena that owns every
+device byte, a plugin interface with no workspace, a request path that must
+not allocate), so the library offers this one forward whose scratch lives in a
+static device array.  This test calls both entry points through the C ABI on
+the same inputs, twice in a row with different data (the static scratch keeps
+the previous call's contents), and checks that the outputs agree within the
+tolerance the parity tests use.  It runs on its own in a fresh process as well
+as after the other tests; its file name makes pytest collect it last.
+"""
+
+import ctypes
+
+import pytest
+import torch
+
+from gemm_epilogue_fusion_tmem_b200 import synth
+from tests.parity import assert_rel, assert_tol
+
+pytestmark = pytest.mark.gpu
+
+
+def _static_fwd(lib, t, H, r, Y, AB, M, K, d, N, eps):
+    fn = lib.coda_grg_fwd_prefolded_static
+    P = ctypes.c_void_p
+    fn.restype = ctypes.c_int
+    fn.argtypes = [P] * 8 + [ctypes.c_int] * 4 + [ctypes.c_float, P]
+    ptr = lambda x: ctypes.c_void_p(x.data_ptr())
+    return fn(ptr(t["X"]), ptr(t["W1"]), ptr(t["R"]), ptr(t["W2g"]), ptr(H), ptr(r), ptr(Y), ptr(AB),
+              M, K, d, N, ctypes.c_float(eps), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+
+
+def test_static_scratch_forward_matches_workspace_forward(cuda_lib):
+    lib = cuda_lib.library()
+    M, K, d, F, eps = 520, 512, 768, 640, 1e-6   # ragged rows and a ragged partial-RMS tile
+    N = 2 * F
+    for seed in (11, 12):  # two calls in a row share the static scratch
+        t = {k: v.cuda() for k, v in synth.grg_inputs(M, K, d, F, seed=seed).items()}
+        t["W2g"] = cuda_lib.fold_gain(t["W2"], t["g"])
+        ref = cuda_lib.grg_fwd(t["X"], t["W1"], t["R"], t["g"], t["W2"], eps, W2g=t["W2g"])
+        H = torch.full((M, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+        r = torch.full((M,), float("nan"), dtype=torch.float32, device="cuda")
+        Y = torch.full((M, F), float("nan"), dtype=torch.bfloat16, device="cuda")
+        AB = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        st = _static_fwd(lib, t, H, r, Y, AB, M, K, d, N, eps)
+        assert st == 0, f"coda_grg_fwd_prefolded_static returned {st}"
+        torch.cuda.synchronize()
+        assert_tol(H, ref["H"].double().cpu().numpy(), f"static H seed {seed}")
+        assert_rel(r, ref["r"].double().cpu().numpy(), f"static r seed {seed}")
+        assert_tol(Y, ref["Y"].double().cpu().numpy(), f"static Y seed {seed}")
+        assert_tol(AB, ref["AB"].double().cpu().numpy(), f"static AB seed {seed}")
+
+
+def test_static_scratch_forward_rejects_oversized_shapes(cuda_lib):
+    lib = cuda_lib.library()
+    fn = lib.coda_grg_fwd_prefolded_static
+    P = ctypes.c_void_p
+    fn.restype = ctypes.c_int
+    fn.argtypes = [P] * 8 + [ctypes.c_int] * 4 + [ctypes.c_float, P]
+    one = ctypes.c_void_p(256)
+    # M * ceil(d/256) = 40000 * 32 > 2^20 partial sums: CODA_ERR_WORKSPACE_TOO_SMALL (4), nothing enqueued.
+    assert fn(one, one, one, one, one, one, one, one, 40000, 64, 8192, 128, ctypes.c_float(1e-6), None) == 4
