@@ -6,6 +6,7 @@
 #include <algorithm>
 #include <atomic>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 
 #include "coda.h"
@@ -24,10 +25,12 @@ inline int cdiv(long long a, long long b) { return (int)((a + b - 1) / b); }
 
 // ------------------------------------------------------------------ device checks
 
+constexpr int kKernelSlots = 48;  // (EPI, A major, B major, pair) instantiations
 struct DevInfo {
   int num_sms = 0;
   int major = 0;
-  bool smem_set[16] = {};
+  bool configured[kKernelSlots] = {};
+  int max_clusters[kKernelSlots] = {};
 };
 DevInfo g_dev[64];
 
@@ -87,34 +90,74 @@ bool make_operand_map(CUtensorMap* m, const void* base, long long mn, long long 
 
 // ------------------------------------------------------------------ GEMM launch
 
-template <int EPI, bool A_MN, bool B_MN>
-coda_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, GemmParams p, cudaStream_t s) {
+// CTA-pair (cta_group::2, 256-row tiles) is the default GEMM mode; setting
+// the environment variable CODA_CTA_PAIR=0 selects one 128-row tile per CTA.
+bool use_pair() {
+  static const bool v = [] {
+    const char* e = std::getenv("CODA_CTA_PAIR");
+    return !(e != nullptr && e[0] == '0');
+  }();
+  return v;
+}
+inline int tile_m(bool pair) { return pair ? 256 : 128; }
+
+template <int EPI, bool A_MN, bool B_MN, bool PAIR>
+coda_status launch_gemm_mode(const CUtensorMap& ta, const CUtensorMap& tb, GemmParams p, cudaStream_t s) {
+  using C = TileCfg<PAIR>;
   int dev = 0;
   coda_status st = current_device(dev);
   if (st != CODA_OK) return st;
-  auto kern = gemm_tc_kernel<EPI, A_MN, B_MN>;
-  const int slot = EPI * 4 + (A_MN ? 2 : 0) + (B_MN ? 1 : 0);
-  if (!g_dev[dev].smem_set[slot]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES) != cudaSuccess)
+  auto kern = gemm_tc_kernel<EPI, A_MN, B_MN, PAIR>;
+  const int slot = ((EPI * 4 + (A_MN ? 2 : 0) + (B_MN ? 1 : 0)) * 2) + (PAIR ? 1 : 0);
+  DevInfo& di = g_dev[dev];
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = C::CTAS;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = PAIR ? 1 : 0;
+  if (!di.configured[slot]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
       return CODA_ERR_CUDA;
-    g_dev[dev].smem_set[slot] = true;
+    int clusters = di.num_sms / C::CTAS;
+    if (PAIR) {
+      cfg.gridDim = dim3(2 * clusters, 1, 1);
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n > 0) clusters = std::min(clusters, n);
+    }
+    di.max_clusters[slot] = clusters;
+    di.configured[slot] = true;
   }
   p.kernel_id = (uint32_t)(slot + 1);
   p.wait_limit_ns = g_wait_limit_ns.load();
   const int tiles = p.num_m_tiles * p.num_n_tiles;
-  const int grid = std::min(tiles, g_dev[dev].num_sms);
-  if (grid <= 0) return CODA_OK;
-  kern<<<grid, NUM_THREADS, GEMM_SMEM_BYTES, s>>>(ta, tb, p);
+  const int units = std::min(tiles, di.max_clusters[slot]);  // persistent: one tile stream per CTA (pair)
+  if (units <= 0) return CODA_OK;
+  cfg.gridDim = dim3(units * C::CTAS, 1, 1);
+  if (cudaLaunchKernelEx(&cfg, kern, ta, tb, p) != cudaSuccess) return CODA_ERR_CUDA;
   return cudaPeekAtLastError() == cudaSuccess ? CODA_OK : CODA_ERR_CUDA;
 }
 
-GemmParams base_params(int M, int N, int K, int tile_n, void* ws) {
+template <int EPI, bool A_MN, bool B_MN>
+coda_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, cudaStream_t s,
+                        bool pair) {
+  return pair ? launch_gemm_mode<EPI, A_MN, B_MN, true>(ta, tb, p, s)
+              : launch_gemm_mode<EPI, A_MN, B_MN, false>(ta, tb, p, s);
+}
+
+GemmParams base_params(int M, int N, int K, int tile_n, void* ws, bool pair) {
   GemmParams p;
   std::memset(&p, 0, sizeof(p));
   p.M = M;
   p.N = N;
   p.K = K;
-  p.num_m_tiles = cdiv(M, BM);
+  p.num_m_tiles = cdiv(M, tile_m(pair));
   p.num_n_tiles = cdiv(N, tile_n);
   p.k_blocks = cdiv(K, BK);
   p.status = static_cast<uint32_t*>(ws);
@@ -127,17 +170,18 @@ inline const __nv_bfloat16* cbf(const void* p) { return static_cast<const __nv_b
 // Plain C = op(A) op(B)^T with the EPI_STORE epilogue (optional column scale).
 coda_status gemm_store(const void* A, const void* B, void* C, int M, int N, int K, bool a_mn, bool b_mn,
                        const void* colscale, void* ws, cudaStream_t s) {
+  const bool pair = use_pair();
   CUtensorMap ta, tb;
-  if (!make_operand_map(&ta, A, M, K, a_mn, BM) || !make_operand_map(&tb, B, N, K, b_mn, BN))
+  if (!make_operand_map(&ta, A, M, K, a_mn, BM) || !make_operand_map(&tb, B, N, K, b_mn, pair ? BN / 2 : BN))
     return CODA_ERR_CUDA;
-  GemmParams p = base_params(M, N, K, BN, ws);
+  GemmParams p = base_params(M, N, K, BN, ws, pair);
   p.out = bf(C);
   p.ldo = N;
   p.colvec = cbf(colscale);
-  if (!a_mn && !b_mn) return launch_gemm<EPI_STORE, false, false>(ta, tb, p, s);
-  if (!a_mn && b_mn) return launch_gemm<EPI_STORE, false, true>(ta, tb, p, s);
-  if (a_mn && b_mn) return launch_gemm<EPI_STORE, true, true>(ta, tb, p, s);
-  return launch_gemm<EPI_STORE, true, false>(ta, tb, p, s);
+  if (!a_mn && !b_mn) return launch_gemm<EPI_STORE, false, false>(ta, tb, p, s, pair);
+  if (!a_mn && b_mn) return launch_gemm<EPI_STORE, false, true>(ta, tb, p, s, pair);
+  if (a_mn && b_mn) return launch_gemm<EPI_STORE, true, true>(ta, tb, p, s, pair);
+  return launch_gemm<EPI_STORE, true, false>(ta, tb, p, s, pair);
 }
 
 coda_status launch_status(cudaError_t e) { return e == cudaSuccess ? CODA_OK : CODA_ERR_CUDA; }
@@ -148,14 +192,15 @@ coda_status gemm_swiglu(const void* A, const void* Wgu, const float* r, void* Y,
   CUtensorMap ta, tb;
   if (!make_operand_map(&ta, A, M, K, false, BM) || !make_operand_map(&tb, Wgu, 2LL * F, K, false, BN / 2))
     return CODA_ERR_CUDA;
-  GemmParams p = base_params(M, F, K, BN / 2, ws);
+  const bool pair = use_pair();
+  GemmParams p = base_params(M, F, K, BN / 2, ws, pair);
   p.split = F;
   p.out = bf(Y);
   p.ldo = F;
   p.out2 = bf(AB);
   p.ldo2 = 2 * F;
   p.rowvec = r;
-  return launch_gemm<EPI_SWIGLU, false, false>(ta, tb, p, s);
+  return launch_gemm<EPI_SWIGLU, false, false>(ta, tb, p, s, pair);
 }
 
 }  // namespace
@@ -313,17 +358,18 @@ coda_status coda_grg_fwd(const void* X, const void* W1, const void* R, const voi
 
   // GEMM1 + residual + partial sums of squares.
   {
+    const bool pair = use_pair();
     CUtensorMap ta, tb;
-    if (!make_operand_map(&ta, X, M, K, false, BM) || !make_operand_map(&tb, W1, d, K, false, BN))
+    if (!make_operand_map(&ta, X, M, K, false, BM) || !make_operand_map(&tb, W1, d, K, false, pair ? BN / 2 : BN))
       return CODA_ERR_CUDA;
-    GemmParams p = base_params(M, d, K, BN, ws);
+    GemmParams p = base_params(M, d, K, BN, ws, pair);
     p.out = bf(H);
     p.ldo = d;
     p.in0 = cbf(R);
     p.ld_in0 = d;
     p.part = P;
     p.ld_part = T;
-    CODA_TRY((launch_gemm<EPI_RESID_RMS, false, false>(ta, tb, p, s)));
+    CODA_TRY((launch_gemm<EPI_RESID_RMS, false, false>(ta, tb, p, s, pair)));
   }
   // Row reduce -> r.
   rms_rowreduce_kernel<<<cdiv(M, 256), 256, 0, s>>>(P, T, r, M, 1.0f / (float)d, eps);
@@ -345,7 +391,7 @@ BwdWs bwd_ws(int M, int d, int N) {
   w.dap_off = kStatusBytes;
   w.c_off = align_up(w.dap_off + (size_t)M * N * 2, 256);
   w.pg_off = align_up(w.c_off + (size_t)M * 4, 256);
-  w.pg_rows = cdiv(M, BM) * 4;
+  w.pg_rows = cdiv(M, 256) * 8;  // enough for either tile height
   w.total = align_up(w.pg_off + (size_t)w.pg_rows * d * 4, 256);
   return w;
 }
@@ -378,6 +424,7 @@ coda_status coda_grg_bwd(const void* dY, const void* dH_in_or_null, const void* 
   float* Pg = reinterpret_cast<float*>(wsb + w.pg_off);
   const int F = N / 2;
 
+  const bool pair = use_pair();
   // SwiGLU backward + RMSNorm row statistic.
   swiglu_bwd_rowstat_kernel<<<M, ROWSTAT_THREADS, 0, s>>>(cbf(dY), cbf(AB), r, dAp, cvec, F, 1.0f / (float)d);
   CODA_TRY(launch_status(cudaPeekAtLastError()));
@@ -386,7 +433,7 @@ coda_status coda_grg_bwd(const void* dY, const void* dH_in_or_null, const void* 
     CUtensorMap ta, tb;
     if (!make_operand_map(&ta, dAp, M, N, false, BM) || !make_operand_map(&tb, W2, d, N, true, BN))
       return CODA_ERR_CUDA;
-    GemmParams p = base_params(M, d, N, BN, ws);
+    GemmParams p = base_params(M, d, N, BN, ws, pair);
     p.out = bf(dR);
     p.ldo = d;
     p.in0 = cbf(H);
@@ -396,9 +443,10 @@ coda_status coda_grg_bwd(const void* dY, const void* dH_in_or_null, const void* 
     p.rowvec = cvec;
     p.part = Pg;
     p.ld_part = d;
-    CODA_TRY((launch_gemm<EPI_DN, false, true>(ta, tb, p, s)));
+    CODA_TRY((launch_gemm<EPI_DN, false, true>(ta, tb, p, s, pair)));
   }
-  col_reduce_kernel<<<cdiv(d, 256), 256, 0, s>>>(Pg, w.pg_rows, d, dg);
+  // One partial row per 32 output rows of every (possibly partial) row tile.
+  col_reduce_kernel<<<cdiv(d, 256), 256, 0, s>>>(Pg, cdiv(M, tile_m(pair)) * tile_m(pair) / 32, d, dg);
   CODA_TRY(launch_status(cudaPeekAtLastError()));
   // dW2 = g * (dA'^T H).
   CODA_TRY(gemm_store(dAp, H, dW2, N, d, M, true, true, g, ws, s));
@@ -462,13 +510,14 @@ coda_status coda_swiglu_bwd(const void* dOut, const void* X, const void* Wgu, co
     CUtensorMap ta, tb;
     if (!make_operand_map(&ta, dOut, M, d, false, BM) || !make_operand_map(&tb, Wdown, F, d, true, BN))
       return CODA_ERR_CUDA;
-    GemmParams p = base_params(M, F, d, BN, ws);
+    const bool pair = use_pair();
+    GemmParams p = base_params(M, F, d, BN, ws, pair);
     p.split = F;
     p.out = dA;
     p.ldo = 2 * F;
     p.in0 = cbf(AB);
     p.ld_in0 = 2 * F;
-    CODA_TRY((launch_gemm<EPI_SWIGLU_BWD, false, true>(ta, tb, p, s)));
+    CODA_TRY((launch_gemm<EPI_SWIGLU_BWD, false, true>(ta, tb, p, s, pair)));
   }
   CODA_TRY(gemm_store(dOut, Y, dWdown, d, F, M, true, true, nullptr, ws, s));
   CODA_TRY(gemm_store(dA, X, dWgu, 2 * F, d, M, true, true, nullptr, ws, s));
@@ -527,17 +576,18 @@ extern "C" coda_status coda_grg_fwd_prefolded_static(const void* X, const void* 
   float* P = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + kStatusBytes);
   const int F = N / 2;
   {
+    const bool pair = use_pair();
     CUtensorMap ta, tb;
-    if (!make_operand_map(&ta, X, M, K, false, BM) || !make_operand_map(&tb, W1, d, K, false, BN))
+    if (!make_operand_map(&ta, X, M, K, false, BM) || !make_operand_map(&tb, W1, d, K, false, pair ? BN / 2 : BN))
       return CODA_ERR_CUDA;
-    GemmParams p = base_params(M, d, K, BN, scratch);
+    GemmParams p = base_params(M, d, K, BN, scratch, pair);
     p.out = bf(H);
     p.ldo = d;
     p.in0 = cbf(R);
     p.ld_in0 = d;
     p.part = P;
     p.ld_part = T;
-    CODA_TRY((launch_gemm<EPI_RESID_RMS, false, false>(ta, tb, p, s)));
+    CODA_TRY((launch_gemm<EPI_RESID_RMS, false, false>(ta, tb, p, s, pair)));
   }
   rms_rowreduce_kernel<<<cdiv(M, 256), 256, 0, s>>>(P, T, r, M, 1.0f / (float)d, eps);
   CODA_TRY(launch_status(cudaPeekAtLastError()));

@@ -27,15 +27,10 @@ namespace coda {
 constexpr int BM = 128;              // tile rows (TMEM lanes)
 constexpr int BN = 256;              // tile columns (TMEM columns per accumulator)
 constexpr int BK = 64;               // reduction depth per stage (128 bytes of bf16)
-constexpr int STAGES = 4;
 constexpr int UMMA_K = 16;
-constexpr int A_STAGE_BYTES = BM * BK * 2;  // 16 KiB
-constexpr int B_STAGE_BYTES = BN * BK * 2;  // 32 KiB
-constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
 constexpr int MN_CHUNK_BYTES = 64 * BK * 2;  // one [64 k][64 mn] MN-major chunk, 8 KiB
 constexpr int NUM_THREADS = 192;
 constexpr uint32_t TMEM_COLS = 2 * BN;
-constexpr int GEMM_SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 constexpr int GROUP_M = 16;          // tile rasterisation: 16 row tiles per group
 
 enum Epi : int {
@@ -118,9 +113,11 @@ __device__ __forceinline__ void warp_column_sums(float (&v)[32], int lane) {
 
 __device__ __forceinline__ float sigmoid_f(float x) { return __frcp_rn(1.0f + __expf(-x)); }
 
+// One 128-row half-tile of the epilogue: this thread owns output row `row`
+// (valid when rv), `group32` = (row - lane) / 32 indexes the per-warp partials.
 template <int EPI>
-__device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbase, int row, bool rv, int m_blk,
-                                              int n_blk, int q, int lane) {
+__device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbase, int row, bool rv, int group32,
+                                              int n_blk, int lane) {
   if constexpr (EPI == EPI_STORE) {
     const int n0 = n_blk * BN;
 #pragma unroll 1
@@ -216,7 +213,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbas
 #pragma unroll
       for (int i = 0; i < 32; ++i) v[i] *= h[i];
       warp_column_sums(v, lane);
-      p.part[(size_t)(m_blk * 4 + q) * p.ld_part + n0 + c + lane] = v[0];
+      p.part[(size_t)group32 * p.ld_part + n0 + c + lane] = v[0];
     }
   } else if constexpr (EPI == EPI_SWIGLU_BWD) {
     const int n0 = n_blk * BN;
@@ -246,17 +243,35 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbas
   }
 }
 
-template <int EPI, bool A_MN, bool B_MN>
+// Per-mode constants.  PAIR = one 256 x 256 tile per CTA pair (cta_group::2:
+// each CTA holds 128 rows of A and half of B, the leader issues M=256 MMAs);
+// otherwise one 128 x 256 tile per CTA.
+template <bool PAIR>
+struct TileCfg {
+  static constexpr int STAGES = PAIR ? 6 : 4;
+  static constexpr int TILE_M = PAIR ? 256 : 128;
+  static constexpr int B_ROWS = PAIR ? 128 : 256;      // B rows (output columns) held per CTA
+  static constexpr int A_BYTES = 128 * BK * 2;         // 16 KiB
+  static constexpr int B_BYTES = B_ROWS * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+  static constexpr int MMA_M = PAIR ? 256 : 128;
+  static constexpr int CTAS = PAIR ? 2 : 1;
+};
+
+template <int EPI, bool A_MN, bool B_MN, bool PAIR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const GemmParams p) {
+  using C = TileCfg<PAIR>;
+  constexpr int S = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
-  uint8_t* sB = smem + STAGES * A_STAGE_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * B_STAGE_BYTES);
-  uint64_t* empty = full + STAGES;
-  uint64_t* tfull = empty + STAGES;
+  uint8_t* sB = smem + S * C::A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + S * C::B_BYTES);
+  uint64_t* empty = full + S;
+  uint64_t* tfull = empty + S;
   uint64_t* tempty = tfull + 2;
   uint64_t* mma_done = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
@@ -264,15 +279,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;  // 0 = the pair's leader
+  const int first_tile = PAIR ? (int)cluster_id_x() : (int)blockIdx.x;
+  const int tile_step = PAIR ? (int)num_clusters_x() : (int)gridDim.x;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 4);
+      mbar_init(&tempty[a], 4 * C::CTAS);  // one arrival per epilogue warp of the pair
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -281,11 +299,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tma_prefetch_desc(&tmB);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_slot, TMEM_COLS);  // same warp and slot in both CTAs
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR) cluster_sync(); else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
@@ -295,41 +318,64 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      // ---------------------------------------------------------------- producer
+      // ---------------------------------------------------------------- producer (every CTA)
       const uint64_t hint = l2_policy_evict_normal();
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      for (int tile = first_tile; tile < num_tiles && ok; tile += tile_step) {
         int m_blk, n_blk;
         tile_coords(tile, p.num_m_tiles, p.num_n_tiles, m_blk, n_blk);
+        const int a_row = m_blk * C::TILE_M + (int)rank * 128;
         for (int kb = 0; kb < p.k_blocks; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, ctl, 0, kWaitEmpty)) {
             ok = false;
             break;
           }
-          uint64_t* bar = &full[stage];
-          mbar_arrive_expect_tx(bar, STAGE_BYTES);
-          uint8_t* a_dst = sA + stage * A_STAGE_BYTES;
-          uint8_t* b_dst = sB + stage * B_STAGE_BYTES;
+          uint8_t* a_dst = sA + stage * C::A_BYTES;
+          uint8_t* b_dst = sB + stage * C::B_BYTES;
           const int k0 = kb * BK;
-          if constexpr (!A_MN) {
-            tma_load_2d(a_dst, &tmA, bar, k0, m_blk * BM, hint);
-          } else {
+          if constexpr (PAIR) {
+            // Both CTAs' bytes complete on the leader's full barrier.
+            if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
+            const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
+            if constexpr (!A_MN) {
+              tma_load_2d_pair(a_dst, &tmA, bar, k0, a_row, hint);
+            } else {
 #pragma unroll
-            for (int c = 0; c < BM / 64; ++c) tma_load_2d(a_dst + c * MN_CHUNK_BYTES, &tmA, bar, m_blk * BM + c * 64, k0, hint);
-          }
-          if constexpr (EPI == EPI_SWIGLU) {
-            tma_load_2d(b_dst, &tmB, bar, k0, n_blk * (BN / 2), hint);
-            tma_load_2d(b_dst + B_STAGE_BYTES / 2, &tmB, bar, k0, p.split + n_blk * (BN / 2), hint);
-          } else if constexpr (!B_MN) {
-            tma_load_2d(b_dst, &tmB, bar, k0, n_blk * BN, hint);
-          } else {
+              for (int c = 0; c < 2; ++c) tma_load_2d_pair(a_dst + c * MN_CHUNK_BYTES, &tmA, bar, a_row + c * 64, k0, hint);
+            }
+            if constexpr (EPI == EPI_SWIGLU) {
+              // Leader holds the 128 gate rows, the peer the 128 up rows of these output columns.
+              tma_load_2d_pair(b_dst, &tmB, bar, k0, (rank ? p.split : 0) + n_blk * (BN / 2), hint);
+            } else if constexpr (!B_MN) {
+              tma_load_2d_pair(b_dst, &tmB, bar, k0, n_blk * BN + (int)rank * 128, hint);
+            } else {
 #pragma unroll
-            for (int c = 0; c < BN / 64; ++c) tma_load_2d(b_dst + c * MN_CHUNK_BYTES, &tmB, bar, n_blk * BN + c * 64, k0, hint);
+              for (int c = 0; c < 2; ++c)
+                tma_load_2d_pair(b_dst + c * MN_CHUNK_BYTES, &tmB, bar, n_blk * BN + (int)rank * 128 + c * 64, k0, hint);
+            }
+          } else {
+            uint64_t* bar = &full[stage];
+            mbar_arrive_expect_tx(bar, C::STAGE_BYTES);
+            if constexpr (!A_MN) {
+              tma_load_2d(a_dst, &tmA, bar, k0, a_row, hint);
+            } else {
+#pragma unroll
+              for (int c = 0; c < 2; ++c) tma_load_2d(a_dst + c * MN_CHUNK_BYTES, &tmA, bar, a_row + c * 64, k0, hint);
+            }
+            if constexpr (EPI == EPI_SWIGLU) {
+              tma_load_2d(b_dst, &tmB, bar, k0, n_blk * (BN / 2), hint);
+              tma_load_2d(b_dst + C::B_BYTES / 2, &tmB, bar, k0, p.split + n_blk * (BN / 2), hint);
+            } else if constexpr (!B_MN) {
+              tma_load_2d(b_dst, &tmB, bar, k0, n_blk * BN, hint);
+            } else {
+#pragma unroll
+              for (int c = 0; c < BN / 64; ++c) tma_load_2d(b_dst + c * MN_CHUNK_BYTES, &tmB, bar, n_blk * BN + c * 64, k0, hint);
+            }
           }
           ++issued;
-          if (++stage == STAGES) {
+          if (++stage == S) {
             stage = 0;
             phase ^= 1u;
           }
@@ -337,15 +383,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------------------------------------------------------- MMA issuer
-      constexpr uint32_t idesc = make_idesc_bf16(BM, BN, A_MN, B_MN);
+    if (lane == 0 && rank == 0) {
+      // ---------------------------------------------------------------- MMA issuer (pair leader)
+      constexpr uint32_t idesc = make_idesc_bf16(C::MMA_M, BN, A_MN, B_MN);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      for (int tile = first_tile; tile < num_tiles && ok; tile += tile_step) {
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, ctl, 1, kWaitAccEmpty)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
@@ -355,8 +401,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t a_base = smem_u32(sA + stage * A_STAGE_BYTES);
-          const uint32_t b_base = smem_u32(sB + stage * B_STAGE_BYTES);
+          const uint32_t a_base = smem_u32(sA + stage * C::A_BYTES);
+          const uint32_t b_base = smem_u32(sB + stage * C::B_BYTES);
 #pragma unroll
           for (int k = 0; k < BK / UMMA_K; ++k) {
             // K-major: advance 16 elements (32 B) inside the 128-B swizzled row;
@@ -365,29 +411,43 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                      : make_sdesc_sw128(a_base + k * 32, 16, 1024);
             const uint64_t bd = B_MN ? make_sdesc_sw128(b_base + k * 2048, MN_CHUNK_BYTES, 1024)
                                      : make_sdesc_sw128(b_base + k * 32, 16, 1024);
-            umma_bf16(d_tmem, ad, bd, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+            if constexpr (PAIR) umma_bf16_pair(d_tmem, ad, bd, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+            else umma_bf16(d_tmem, ad, bd, idesc, (kb > 0 || k > 0) ? 1u : 0u);
           }
-          umma_commit(&empty[stage]);  // frees the stage once these MMAs have read it
-          if (++stage == STAGES) {
+          // Free the stage (in both CTAs of a pair) once these MMAs have read it.
+          if constexpr (PAIR) {
+            umma_commit_pair(mapa_shared(smem_u32(&empty[stage]), 0));
+            umma_commit_pair(mapa_shared(smem_u32(&empty[stage]), 1));
+          } else {
+            umma_commit(&empty[stage]);
+          }
+          if (++stage == S) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        umma_commit(&tfull[acc]);  // accumulator ready for the epilogue
+        // Accumulator ready for the epilogue warps (of both CTAs of a pair).
+        if constexpr (PAIR) {
+          umma_commit_pair(mapa_shared(smem_u32(&tfull[acc]), 0));
+          umma_commit_pair(mapa_shared(smem_u32(&tfull[acc]), 1));
+        } else {
+          umma_commit(&tfull[acc]);
+        }
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
       }
       // Every MMA issued by this thread has completed once mma_done fires.
-      umma_commit(mma_done);
+      if constexpr (PAIR) umma_commit_pair(mapa_shared(smem_u32(mma_done), 0));
+      else umma_commit(mma_done);
       mbar_wait(mma_done, 0, ctl, 1, kWaitDrain);
     }
   } else {
-    // ---------------------------------------------------------------- epilogue
+    // ---------------------------------------------------------------- epilogue (every CTA)
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+    for (int tile = first_tile; tile < num_tiles; tile += tile_step) {
       int m_blk, n_blk;
       tile_coords(tile, p.num_m_tiles, p.num_n_tiles, m_blk, n_blk);
       // Warp-uniform outcome: tcgen05.ld below needs all 32 lanes converged.
@@ -395,35 +455,40 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
-      const int row = m_blk * BM + q * 32 + lane;
-      epilogue_tile<EPI>(p, tbase, row, row < p.M, m_blk, n_blk, q, lane);
+      const int row0 = m_blk * C::TILE_M + (int)rank * 128 + q * 32;
+      epilogue_tile<EPI>(p, tbase, row0 + lane, row0 + lane < p.M, row0 / 32, n_blk, lane);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (lane == 0) {
+        if constexpr (PAIR) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));
+        else mbar_arrive(&tempty[acc]);
+      }
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
   }
 
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR) cluster_sync(); else __syncthreads();
   if (*abort_flag) {
-    // A role gave up: let the last (up to STAGES) copies land before the
-    // CTA's shared memory is released.  Every wait here is bounded too.
-    if (warp == 0 && lane == 0) {
-      const int first = issued > STAGES ? issued - STAGES : 0;
+    // A role gave up: let the last (up to STAGES) copies land before shared
+    // memory is released.  Every wait here is bounded too.
+    if (warp == 0 && lane == 0 && rank == 0) {
+      const int first = issued > S ? issued - S : 0;
       for (int i = first; i < issued; ++i) {
-        const uint32_t par = (uint32_t)((i / STAGES) & 1);
+        const uint32_t par = (uint32_t)((i / S) & 1);
         const uint64_t t0 = global_timer_ns();
-        while (!mbar_try_wait(&full[i % STAGES], par) && global_timer_ns() - t0 < ctl.limit_ns) {
+        while (!mbar_try_wait(&full[i % S], par) && global_timer_ns() - t0 < ctl.limit_ns) {
         }
       }
     }
     __syncthreads();
   }
+  if constexpr (PAIR) cluster_sync();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    if constexpr (PAIR) tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    else tmem_dealloc(tmem_base, TMEM_COLS);
   }
 }
 
