@@ -50,6 +50,7 @@ def _args():
     p.add_argument("--workload", choices=sorted(WORKLOADS), default="7B")
     p.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed oracle sample")
     p.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
+    p.add_argument("--no-unfused", action="store_true", help="skip timing the unfused comparison sequence")
     return p.parse_args()
 
 
@@ -278,6 +279,30 @@ def _make_step(kind, s, bwd, dev):
     return step, outs, 6, ["Out", "dX", "dWgu", "dWdown"], ws
 
 
+def _make_unfused_step(s, bwd, dev):
+    """The same block run operator by operator (every intermediate in HBM)."""
+    import torch
+    from gemm_epilogue_fusion_tmem_b200 import binding as B
+    lib = B.library()
+    M, K, d, F = s["M"], s["K"], s["d"], s["F"]
+    N = 2 * F
+    ws = B.Workspace(max(lib.coda_grg_fwd_unfused_workspace_bytes(M, K, d, N),
+                         lib.coda_grg_bwd_unfused_workspace_bytes(M, K, d, N)), dev["X"].device)
+    fo = B.grg_fwd_unfused(dev["X"], dev["W1"], dev["R"], dev["g"], dev["W2"], s["eps"], ws=ws)
+    bo = {}
+    if bwd:
+        bo = B.grg_bwd_unfused(dev["dY"], dev["X"], dev["W1"], fo["H"], fo["r"], fo["AB"], fo["U"], dev["g"],
+                               dev["W2"], ws=ws)
+
+    def step():
+        B.grg_fwd_unfused(dev["X"], dev["W1"], dev["R"], dev["g"], dev["W2"], s["eps"], out=fo, ws=ws)
+        if bwd:
+            B.grg_bwd_unfused(dev["dY"], dev["X"], dev["W1"], fo["H"], fo["r"], fo["AB"], fo["U"], dev["g"],
+                              dev["W2"], out=bo, ws=ws)
+
+    return step, (13 if bwd else 5), ws
+
+
 def _dominant_kernel(kind, s, dev, outs, reps=20):
     """Time the dominant kernel alone: the gate/up GEMM with the r + SwiGLU epilogue."""
     import torch
@@ -353,6 +378,31 @@ def run_coda(a):
     ms_max = float(t.item())
     value = flops * a.steps * world / (ms_max / 1e3) / 1e12
 
+    # The unfused comparison sequence, timed the same way right after.
+    unfused = None
+    if kind == "grg" and not a.no_unfused:
+        ustep, ulaunch, uws = _make_unfused_step(s, bwd, dev)
+        for _ in range(max(a.warmup, 3)):
+            ustep()
+        torch.cuda.synchronize()
+        barrier()
+        e0.record(st)
+        for _ in range(a.steps):
+            ustep()
+        e1.record(st)
+        torch.cuda.synchronize()
+        barrier()
+        tu = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=device)
+        if world > 1:
+            dist.all_reduce(tu, op=dist.ReduceOp.MAX)
+        u_ms = float(tu.item())
+        unfused = {"ms_per_step": round(u_ms / a.steps, 4),
+                   "value": round(flops * a.steps * world / (u_ms / 1e3) / 1e12, 2), "unit": "TFLOP/s",
+                   "fused_speedup": round(u_ms / ms_max, 4), "gpu_launches_per_step": ulaunch,
+                   "what": "same GEMM kernels with plain stores; residual add, RMSNorm, SwiGLU and their backward "
+                           "as separate HBM-round-trip kernels"}
+        del uws
+
     # Dominant kernel alone (roofline).
     peaks, peaks_src = _peaks()
     kname, k_ms, k_flops = _dominant_kernel(kind, s, dev, outs)
@@ -419,6 +469,7 @@ def run_coda(a):
                        "flops_per_step": flops, "frac_of_sustained_bf16_peak": round(frac_step, 4)},
             "roofline": roofline,
             "cpu_baseline": cpu,
+            "unfused": unfused,
             "e2e": e2e,
             "gpu_launches": launches * a.steps,
             "clocks": clk.summary(),

@@ -67,6 +67,10 @@ def library() -> ctypes.CDLL:
             "coda_swiglu_fwd": (I, [P, P, P, P, P, P, I, I, I, P, S, P]),
             "coda_swiglu_bwd_workspace_bytes": (S, [I, I, I]),
             "coda_swiglu_bwd": (I, [P, P, P, P, P, P, P, P, P, I, I, I, P, S, P]),
+            "coda_grg_fwd_unfused_workspace_bytes": (S, [I, I, I, I]),
+            "coda_grg_fwd_unfused": (I, [P] * 10 + [I, I, I, I, F, P, S, P]),
+            "coda_grg_bwd_unfused_workspace_bytes": (S, [I, I, I, I]),
+            "coda_grg_bwd_unfused": (I, [P] * 15 + [I, I, I, I, P, S, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)
@@ -178,9 +182,11 @@ def gemm_swiglu(A, Wgu, r=None, save_ab: bool = True, out: dict | None = None,
     if r is not None:
         _req(r, "r", torch.float32, (M,))
     o = dict(out or {})
-    o.setdefault("Y", torch.empty(M, F, dtype=torch.bfloat16, device=A.device))
+    if "Y" not in o:
+        o["Y"] = torch.empty(M, F, dtype=torch.bfloat16, device=A.device)
     if save_ab:
-        o.setdefault("AB", torch.empty(M, 2 * F, dtype=torch.bfloat16, device=A.device))
+        if "AB" not in o:
+            o["AB"] = torch.empty(M, 2 * F, dtype=torch.bfloat16, device=A.device)
     ws = ws or workspace(lib.coda_gemm_workspace_bytes(), A.device)
     _check(lib.coda_gemm_swiglu(_ptr(A), _ptr(Wgu), _ptr(r), _ptr(o["Y"]), _ptr(o.get("AB") if save_ab else None),
                                 M, K, F, ws.ptr(), ws.nbytes, _stream()), "coda_gemm_swiglu")
@@ -212,11 +218,14 @@ def grg_fwd(X, W1, R, g, W2, eps: float, W2g=None, save_ab: bool = True, out: di
         _req(W2g, "W2g", shape=(N, d))
     o = dict(out or {})
     dev = X.device
-    o.setdefault("H", torch.empty(M, d, dtype=torch.bfloat16, device=dev))
-    o.setdefault("r", torch.empty(M, dtype=torch.float32, device=dev))
-    o.setdefault("Y", torch.empty(M, F, dtype=torch.bfloat16, device=dev))
-    if save_ab:
-        o.setdefault("AB", torch.empty(M, N, dtype=torch.bfloat16, device=dev))
+    if "H" not in o:
+        o["H"] = torch.empty(M, d, dtype=torch.bfloat16, device=dev)
+    if "r" not in o:
+        o["r"] = torch.empty(M, dtype=torch.float32, device=dev)
+    if "Y" not in o:
+        o["Y"] = torch.empty(M, F, dtype=torch.bfloat16, device=dev)
+    if save_ab and "AB" not in o:
+        o["AB"] = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
     _req(o["H"], "H", shape=(M, d)), _req(o["r"], "r", torch.float32, (M,)), _req(o["Y"], "Y", shape=(M, F))
     AB = o.get("AB") if save_ab else None
     if AB is not None:
@@ -243,11 +252,11 @@ def grg_bwd(dY, X, W1, H, r, AB, g, W2, dH_in=None, out: dict | None = None, ws:
         _req(dH_in, "dH_in", shape=(M, d))
     o = dict(out or {})
     dev = X.device
-    o.setdefault("dX", torch.empty(M, K, dtype=torch.bfloat16, device=dev))
-    o.setdefault("dR", torch.empty(M, d, dtype=torch.bfloat16, device=dev))
-    o.setdefault("dW1", torch.empty(d, K, dtype=torch.bfloat16, device=dev))
-    o.setdefault("dW2", torch.empty(N, d, dtype=torch.bfloat16, device=dev))
-    o.setdefault("dg", torch.empty(d, dtype=torch.float32, device=dev))
+    for k, shape, dt in (("dX", (M, K), torch.bfloat16), ("dR", (M, d), torch.bfloat16),
+                         ("dW1", (d, K), torch.bfloat16), ("dW2", (N, d), torch.bfloat16),
+                         ("dg", (d,), torch.float32)):
+        if k not in o:
+            o[k] = torch.empty(*shape, dtype=dt, device=dev)
     ws = ws or workspace(lib.coda_grg_bwd_workspace_bytes(M, K, d, N), dev)
     _check(lib.coda_grg_bwd(_ptr(dY), _ptr(dH_in), _ptr(X), _ptr(W1), _ptr(H), _ptr(r), _ptr(AB), _ptr(g),
                             _ptr(W2), _ptr(o["dX"]), _ptr(o["dR"]), _ptr(o["dW1"]), _ptr(o["dW2"]), _ptr(o["dg"]),
@@ -263,10 +272,13 @@ def swiglu_fwd(X, Wgu, Wdown, save_ab: bool = True, out: dict | None = None, ws:
     _req(X, "X"), _req(Wgu, "Wgu", shape=(2 * F, d)), _req(Wdown, "Wdown", shape=(d, F))
     o = dict(out or {})
     dev = X.device
-    o.setdefault("Y", torch.empty(M, F, dtype=torch.bfloat16, device=dev))
+    if "Y" not in o:
+        o["Y"] = torch.empty(M, F, dtype=torch.bfloat16, device=dev)
     if save_ab:
-        o.setdefault("AB", torch.empty(M, 2 * F, dtype=torch.bfloat16, device=dev))
-    o.setdefault("Out", torch.empty(M, d, dtype=torch.bfloat16, device=dev))
+        if "AB" not in o:
+            o["AB"] = torch.empty(M, 2 * F, dtype=torch.bfloat16, device=dev)
+    if "Out" not in o:
+        o["Out"] = torch.empty(M, d, dtype=torch.bfloat16, device=dev)
     ws = ws or workspace(lib.coda_swiglu_fwd_workspace_bytes(M, d, F), dev)
     _check(lib.coda_swiglu_fwd(_ptr(X), _ptr(Wgu), _ptr(Wdown), _ptr(o["Y"]), _ptr(o.get("AB") if save_ab else None),
                                _ptr(o["Out"]), M, d, F, ws.ptr(), ws.nbytes, _stream()), "coda_swiglu_fwd")
@@ -282,11 +294,67 @@ def swiglu_bwd(dOut, X, Wgu, Wdown, Y, AB, out: dict | None = None, ws: Workspac
     _req(Wdown, "Wdown", shape=(d, F)), _req(Y, "Y", shape=(M, F)), _req(AB, "AB", shape=(M, 2 * F))
     o = dict(out or {})
     dev = X.device
-    o.setdefault("dX", torch.empty(M, d, dtype=torch.bfloat16, device=dev))
-    o.setdefault("dWgu", torch.empty(2 * F, d, dtype=torch.bfloat16, device=dev))
-    o.setdefault("dWdown", torch.empty(d, F, dtype=torch.bfloat16, device=dev))
+    if "dX" not in o:
+        o["dX"] = torch.empty(M, d, dtype=torch.bfloat16, device=dev)
+    if "dWgu" not in o:
+        o["dWgu"] = torch.empty(2 * F, d, dtype=torch.bfloat16, device=dev)
+    if "dWdown" not in o:
+        o["dWdown"] = torch.empty(d, F, dtype=torch.bfloat16, device=dev)
     ws = ws or workspace(lib.coda_swiglu_bwd_workspace_bytes(M, d, F), dev)
     _check(lib.coda_swiglu_bwd(_ptr(dOut), _ptr(X), _ptr(Wgu), _ptr(Wdown), _ptr(Y), _ptr(AB), _ptr(o["dX"]),
                                _ptr(o["dWgu"]), _ptr(o["dWdown"]), M, d, F, ws.ptr(), ws.nbytes, _stream()),
            "coda_swiglu_bwd")
+    return o
+
+
+# ------------------------------------------------------------------ unfused comparison sequence
+
+def grg_fwd_unfused(X, W1, R, g, W2, eps: float, out: dict | None = None, ws: Workspace | None = None) -> dict:
+    """Operator-by-operator forward (measurement/comparison only); returns H, r, Y, AB, U."""
+    lib = library()
+    M, K = X.shape
+    d = W1.shape[0]
+    N = W2.shape[0]
+    F = N // 2
+    _req(X, "X"), _req(W1, "W1", shape=(d, K)), _req(R, "R", shape=(M, d))
+    _req(g, "g", shape=(d,)), _req(W2, "W2", shape=(N, d))
+    o = dict(out or {})
+    dev = X.device
+    for k, shape, dt in (("H", (M, d), torch.bfloat16), ("r", (M,), torch.float32), ("Y", (M, F), torch.bfloat16),
+                         ("AB", (M, N), torch.bfloat16), ("U", (M, d), torch.bfloat16)):
+        if k not in o:
+            o[k] = torch.empty(*shape, dtype=dt, device=dev)
+        _req(o[k], k, dt, shape)
+    ws = ws or workspace(lib.coda_grg_fwd_unfused_workspace_bytes(M, K, d, N), dev)
+    _check(lib.coda_grg_fwd_unfused(_ptr(X), _ptr(W1), _ptr(R), _ptr(g), _ptr(W2), _ptr(o["H"]), _ptr(o["r"]),
+                                    _ptr(o["Y"]), _ptr(o["AB"]), _ptr(o["U"]), M, K, d, N, float(eps),
+                                    ws.ptr(), ws.nbytes, _stream()), "coda_grg_fwd_unfused")
+    return o
+
+
+def grg_bwd_unfused(dY, X, W1, H, r, AB, U, g, W2, dH_in=None, out: dict | None = None,
+                    ws: Workspace | None = None) -> dict:
+    """Operator-by-operator backward (measurement/comparison only); returns dX, dR, dW1, dW2, dg."""
+    lib = library()
+    M, K = X.shape
+    d = W1.shape[0]
+    N = W2.shape[0]
+    F = N // 2
+    _req(dY, "dY", shape=(M, F)), _req(X, "X"), _req(W1, "W1", shape=(d, K)), _req(H, "H", shape=(M, d))
+    _req(r, "r", torch.float32, (M,)), _req(AB, "AB", shape=(M, N)), _req(U, "U", shape=(M, d))
+    _req(g, "g", shape=(d,)), _req(W2, "W2", shape=(N, d))
+    if dH_in is not None:
+        _req(dH_in, "dH_in", shape=(M, d))
+    o = dict(out or {})
+    dev = X.device
+    for k, shape, dt in (("dX", (M, K), torch.bfloat16), ("dR", (M, d), torch.bfloat16),
+                         ("dW1", (d, K), torch.bfloat16), ("dW2", (N, d), torch.bfloat16),
+                         ("dg", (d,), torch.float32)):
+        if k not in o:
+            o[k] = torch.empty(*shape, dtype=dt, device=dev)
+    ws = ws or workspace(lib.coda_grg_bwd_unfused_workspace_bytes(M, K, d, N), dev)
+    _check(lib.coda_grg_bwd_unfused(_ptr(dY), _ptr(dH_in), _ptr(X), _ptr(W1), _ptr(H), _ptr(r), _ptr(AB), _ptr(U),
+                                    _ptr(g), _ptr(W2), _ptr(o["dX"]), _ptr(o["dR"]), _ptr(o["dW1"]), _ptr(o["dW2"]),
+                                    _ptr(o["dg"]), M, K, d, N, ws.ptr(), ws.nbytes, _stream()),
+           "coda_grg_bwd_unfused")
     return o

@@ -12,6 +12,7 @@
 #include "coda.h"
 #include "coda_aux.cuh"
 #include "coda_gemm.cuh"
+#include "coda_unfused.cuh"
 
 namespace coda {
 namespace {
@@ -34,6 +35,9 @@ struct DevInfo {
 };
 DevInfo g_dev[64];
 
+int g_last_sms = 148;
+int num_sms() { return g_last_sms; }
+
 coda_status current_device(int& dev) {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return CODA_ERR_CUDA;
   DevInfo& di = g_dev[dev];
@@ -45,6 +49,7 @@ coda_status current_device(int& dev) {
     di.num_sms = sms;
   }
   if (di.major != 10) return CODA_ERR_NO_SM100;
+  g_last_sms = di.num_sms;
   return CODA_OK;
 }
 
@@ -101,6 +106,75 @@ bool use_pair() {
 }
 inline int tile_m(bool pair) { return pair ? 256 : 128; }
 
+// Programmatic dependent launch between the kernels of a pass (each kernel
+// waits for its predecessor with griddepcontrol.wait before touching global
+// memory); CODA_PDL=0 turns it off.
+bool use_pdl() {
+  static const bool v = [] {
+    const char* e = std::getenv("CODA_PDL");
+    return !(e != nullptr && e[0] == '0');
+  }();
+  return v;
+}
+
+// Launch with the optional cluster size and the PDL attribute.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, int cluster,
+                      Args&&... args) {
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  if (cluster > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  if (use_pdl()) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+// Rasterisation.  Concurrent tiles read the same k-slices at about the same
+// time, so a wave of gm x gn tiles reads gm A tiles and gn B tiles from HBM.
+// The operand with the smaller total is kept resident across waves: its group
+// (row tiles for A, column tiles for B) holds ~32 MiB (CODA_RASTER_MB
+// overrides), and is at least sqrt(concurrent tiles) wide so each wave is
+// close to square; the other operand streams through once per group.
+int raster_budget_mb() {
+  static const int v = [] {
+    const char* e = std::getenv("CODA_RASTER_MB");
+    const int x = e ? std::atoi(e) : 0;
+    return x > 0 ? x : 32;
+  }();
+  return v;
+}
+int pick_group(long long a_rows, long long b_rows, long long K, int num_m, int num_n, bool pair, int num_sms) {
+  const int units = pair ? num_sms / 2 : num_sms;
+  int side = 1;
+  while (side * side < units) ++side;
+  const long long budget = (long long)raster_budget_mb() << 20;
+  if (a_rows <= b_rows) {
+    const long long tile_bytes = (long long)tile_m(pair) * K * 2;
+    const long long g = std::max<long long>(side, budget / std::max(tile_bytes, 1LL));
+    return (int)std::min<long long>(num_m, g);
+  }
+  const long long tile_bytes = (long long)BN * K * 2;
+  const long long g = std::max<long long>(side, budget / std::max(tile_bytes, 1LL));
+  return -(int)std::min<long long>(num_n, g);
+}
+
 template <int EPI, bool A_MN, bool B_MN, bool PAIR>
 coda_status launch_gemm_mode(const CUtensorMap& ta, const CUtensorMap& tb, GemmParams p, cudaStream_t s) {
   using C = TileCfg<PAIR>;
@@ -136,11 +210,13 @@ coda_status launch_gemm_mode(const CUtensorMap& ta, const CUtensorMap& tb, GemmP
   }
   p.kernel_id = (uint32_t)(slot + 1);
   p.wait_limit_ns = g_wait_limit_ns.load();
+  if (p.group_m == 0) p.group_m = 1;
   const int tiles = p.num_m_tiles * p.num_n_tiles;
   const int units = std::min(tiles, di.max_clusters[slot]);  // persistent: one tile stream per CTA (pair)
   if (units <= 0) return CODA_OK;
-  cfg.gridDim = dim3(units * C::CTAS, 1, 1);
-  if (cudaLaunchKernelEx(&cfg, kern, ta, tb, p) != cudaSuccess) return CODA_ERR_CUDA;
+  if (launch_ex(kern, dim3(units * C::CTAS), dim3(NUM_THREADS), C::SMEM_BYTES, s, C::CTAS, ta, tb, p) !=
+      cudaSuccess)
+    return CODA_ERR_CUDA;
   return cudaPeekAtLastError() == cudaSuccess ? CODA_OK : CODA_ERR_CUDA;
 }
 
@@ -175,6 +251,7 @@ coda_status gemm_store(const void* A, const void* B, void* C, int M, int N, int 
   if (!make_operand_map(&ta, A, M, K, a_mn, BM) || !make_operand_map(&tb, B, N, K, b_mn, pair ? BN / 2 : BN))
     return CODA_ERR_CUDA;
   GemmParams p = base_params(M, N, K, BN, ws, pair);
+  p.group_m = pick_group(M, N, K, p.num_m_tiles, p.num_n_tiles, pair, num_sms());
   p.out = bf(C);
   p.ldo = N;
   p.colvec = cbf(colscale);
@@ -194,6 +271,7 @@ coda_status gemm_swiglu(const void* A, const void* Wgu, const float* r, void* Y,
     return CODA_ERR_CUDA;
   const bool pair = use_pair();
   GemmParams p = base_params(M, F, K, BN / 2, ws, pair);
+  p.group_m = pick_group(M, 2LL * F, K, p.num_m_tiles, p.num_n_tiles, pair, num_sms());
   p.split = F;
   p.out = bf(Y);
   p.ldo = F;
@@ -295,8 +373,8 @@ coda_status coda_fold_gain(const void* W2, const void* g, void* W2g, int d, int 
   CODA_TRY(current_device(dev));
   const long long nv = (long long)N * d / 8;
   const int grid = (int)std::min<long long>(cdiv(nv, 256), (long long)g_dev[dev].num_sms * 8);
-  fold_gain_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(cbf(W2), cbf(g), bf(W2g), d, nv);
-  return launch_status(cudaPeekAtLastError());
+  return launch_status(launch_ex(fold_gain_kernel, dim3(grid), dim3(256), 0, static_cast<cudaStream_t>(stream), 1,
+                                 cbf(W2), cbf(g), bf(W2g), d, nv));
 }
 
 // ------------------------------------------------------------------ GRG forward
@@ -363,6 +441,7 @@ coda_status coda_grg_fwd(const void* X, const void* W1, const void* R, const voi
     if (!make_operand_map(&ta, X, M, K, false, BM) || !make_operand_map(&tb, W1, d, K, false, pair ? BN / 2 : BN))
       return CODA_ERR_CUDA;
     GemmParams p = base_params(M, d, K, BN, ws, pair);
+    p.group_m = pick_group(M, d, K, p.num_m_tiles, p.num_n_tiles, pair, num_sms());
     p.out = bf(H);
     p.ldo = d;
     p.in0 = cbf(R);
@@ -372,8 +451,8 @@ coda_status coda_grg_fwd(const void* X, const void* W1, const void* R, const voi
     CODA_TRY((launch_gemm<EPI_RESID_RMS, false, false>(ta, tb, p, s, pair)));
   }
   // Row reduce -> r.
-  rms_rowreduce_kernel<<<cdiv(M, 256), 256, 0, s>>>(P, T, r, M, 1.0f / (float)d, eps);
-  CODA_TRY(launch_status(cudaPeekAtLastError()));
+  CODA_TRY(launch_status(launch_ex(rms_rowreduce_kernel, dim3(cdiv(M, 256)), dim3(256), 0, s, 1, (const float*)P, T,
+                                   r, M, 1.0f / (float)d, eps)));
   // GEMM2 (gate|up) + r scaling + SwiGLU.
   CODA_TRY(gemm_swiglu(H, W2g, r, Y, AB_or_null, M, d, F, ws, s));
   return CODA_OK;
@@ -426,14 +505,15 @@ coda_status coda_grg_bwd(const void* dY, const void* dH_in_or_null, const void* 
 
   const bool pair = use_pair();
   // SwiGLU backward + RMSNorm row statistic.
-  swiglu_bwd_rowstat_kernel<<<M, ROWSTAT_THREADS, 0, s>>>(cbf(dY), cbf(AB), r, dAp, cvec, F, 1.0f / (float)d);
-  CODA_TRY(launch_status(cudaPeekAtLastError()));
+  CODA_TRY(launch_status(launch_ex(swiglu_bwd_rowstat_kernel, dim3(M), dim3(ROWSTAT_THREADS), 0, s, 1, cbf(dY),
+                                   cbf(AB), r, dAp, cvec, F, 1.0f / (float)d)));
   // dn GEMM: dR = g * (dA' W2) - c * H (+ dH_in), with dg column partials.
   {
     CUtensorMap ta, tb;
     if (!make_operand_map(&ta, dAp, M, N, false, BM) || !make_operand_map(&tb, W2, d, N, true, BN))
       return CODA_ERR_CUDA;
     GemmParams p = base_params(M, d, N, BN, ws, pair);
+    p.group_m = pick_group(M, d, N, p.num_m_tiles, p.num_n_tiles, pair, num_sms());
     p.out = bf(dR);
     p.ldo = d;
     p.in0 = cbf(H);
@@ -446,8 +526,8 @@ coda_status coda_grg_bwd(const void* dY, const void* dH_in_or_null, const void* 
     CODA_TRY((launch_gemm<EPI_DN, false, true>(ta, tb, p, s, pair)));
   }
   // One partial row per 32 output rows of every (possibly partial) row tile.
-  col_reduce_kernel<<<cdiv(d, 256), 256, 0, s>>>(Pg, cdiv(M, tile_m(pair)) * tile_m(pair) / 32, d, dg);
-  CODA_TRY(launch_status(cudaPeekAtLastError()));
+  CODA_TRY(launch_status(launch_ex(col_reduce_kernel, dim3(cdiv(d, 256)), dim3(256), 0, s, 1, (const float*)Pg,
+                                   cdiv(M, tile_m(pair)) * tile_m(pair) / 32, d, dg)));
   // dW2 = g * (dA'^T H).
   CODA_TRY(gemm_store(dAp, H, dW2, N, d, M, true, true, g, ws, s));
   // dX = dH W1;  dW1 = dH^T X.
@@ -512,6 +592,7 @@ coda_status coda_swiglu_bwd(const void* dOut, const void* X, const void* Wgu, co
       return CODA_ERR_CUDA;
     const bool pair = use_pair();
     GemmParams p = base_params(M, F, d, BN, ws, pair);
+    p.group_m = pick_group(M, F, d, p.num_m_tiles, p.num_n_tiles, pair, num_sms());
     p.split = F;
     p.out = dA;
     p.ldo = 2 * F;
@@ -522,6 +603,97 @@ coda_status coda_swiglu_bwd(const void* dOut, const void* X, const void* Wgu, co
   CODA_TRY(gemm_store(dOut, Y, dWdown, d, F, M, true, true, nullptr, ws, s));
   CODA_TRY(gemm_store(dA, X, dWgu, 2 * F, d, M, true, true, nullptr, ws, s));
   CODA_TRY(gemm_store(dA, Wgu, dX, M, d, 2 * F, false, true, nullptr, ws, s));
+  return CODA_OK;
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------ unfused comparison sequence
+
+namespace coda {
+namespace {
+inline int ew_grid(long long n_vec8) { return (int)std::min<long long>(cdiv(n_vec8, 256), (long long)num_sms() * 16); }
+}  // namespace
+}  // namespace coda
+
+extern "C" {
+
+size_t coda_grg_fwd_unfused_workspace_bytes(int M, int K, int d, int N) {
+  (void)K, (void)N;
+  if (M < 1 || d < 1) return kStatusBytes;
+  return kStatusBytes + align_up((size_t)M * d * 2, 256);
+}
+
+coda_status coda_grg_fwd_unfused(const void* X, const void* W1, const void* R, const void* g, const void* W2,
+                                 void* H, float* r, void* Y, void* AB, void* U, int M, int K, int d, int N,
+                                 float eps, void* ws, size_t ws_bytes, void* stream) {
+  if (!X || !W1 || !R || !g || !W2 || !H || !r || !Y || !AB || !U || !ws) return CODA_ERR_INVALID_ARG;
+  if (!(eps > 0.f)) return CODA_ERR_INVALID_ARG;
+  CODA_TRY(check_grg_shapes(M, K, d, N));
+  const void* ptrs[] = {X, W1, R, g, W2, H, r, Y, AB, U, ws};
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return CODA_ERR_MISALIGNED;
+  if (ws_bytes < coda_grg_fwd_unfused_workspace_bytes(M, K, d, N)) return CODA_ERR_WORKSPACE_TOO_SMALL;
+  int dev;
+  CODA_TRY(current_device(dev));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  __nv_bfloat16* T = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(ws) + kStatusBytes);
+  const int F = N / 2;
+  CODA_TRY(gemm_store(X, W1, T, M, d, K, false, false, nullptr, ws, s));
+  const long long nh = (long long)M * d / 8;
+  CODA_TRY(launch_status(launch_ex(unf_residual_add_kernel, dim3(ew_grid(nh)), dim3(256), 0, s, 1,
+                                   (const __nv_bfloat16*)T, cbf(R), bf(H), nh)));
+  CODA_TRY(launch_status(launch_ex(unf_rmsnorm_fwd_kernel, dim3(M), dim3(UNF_THREADS), 0, s, 1, cbf(H), cbf(g),
+                                   bf(U), r, d, eps)));
+  CODA_TRY(gemm_store(U, W2, AB, M, N, d, false, false, nullptr, ws, s));
+  const long long ny = (long long)M * F / 8;
+  CODA_TRY(launch_status(launch_ex(unf_swiglu_fwd_kernel, dim3(ew_grid(ny)), dim3(256), 0, s, 1, cbf(AB), bf(Y), F,
+                                   ny)));
+  return CODA_OK;
+}
+
+size_t coda_grg_bwd_unfused_workspace_bytes(int M, int K, int d, int N) {
+  (void)K;
+  if (M < 1 || d < 1 || N < 1) return kStatusBytes;
+  return kStatusBytes + align_up((size_t)M * N * 2, 256) + align_up((size_t)M * d * 2, 256) +
+         align_up((size_t)cdiv(M, UNF_DG_ROWS) * d * 4, 256);
+}
+
+coda_status coda_grg_bwd_unfused(const void* dY, const void* dH_in_or_null, const void* X, const void* W1,
+                                 const void* H, const float* r, const void* AB, const void* U, const void* g,
+                                 const void* W2, void* dX, void* dR, void* dW1, void* dW2, float* dg, int M, int K,
+                                 int d, int N, void* ws, size_t ws_bytes, void* stream) {
+  if (!dY || !X || !W1 || !H || !r || !AB || !U || !g || !W2 || !dX || !dR || !dW1 || !dW2 || !dg || !ws)
+    return CODA_ERR_INVALID_ARG;
+  CODA_TRY(check_grg_shapes(M, K, d, N));
+  const void* ptrs[] = {dY, dH_in_or_null, X, W1, H, r, AB, U, g, W2, dX, dR, dW1, dW2, dg, ws};
+  for (const void* q : ptrs)
+    if (q && !aligned16(q)) return CODA_ERR_MISALIGNED;
+  if (ws_bytes < coda_grg_bwd_unfused_workspace_bytes(M, K, d, N)) return CODA_ERR_WORKSPACE_TOO_SMALL;
+  int dev;
+  CODA_TRY(current_device(dev));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* wsb = static_cast<uint8_t*>(ws) + kStatusBytes;
+  __nv_bfloat16* dA = reinterpret_cast<__nv_bfloat16*>(wsb);
+  wsb += align_up((size_t)M * N * 2, 256);
+  __nv_bfloat16* du = reinterpret_cast<__nv_bfloat16*>(wsb);
+  wsb += align_up((size_t)M * d * 2, 256);
+  float* part = reinterpret_cast<float*>(wsb);
+  const int F = N / 2;
+  const long long ny = (long long)M * F / 8;
+  CODA_TRY(launch_status(launch_ex(unf_swiglu_bwd_kernel, dim3(ew_grid(ny)), dim3(256), 0, s, 1, cbf(dY), cbf(AB),
+                                   dA, F, ny)));
+  CODA_TRY(gemm_store(dA, W2, du, M, d, N, false, true, nullptr, ws, s));
+  CODA_TRY(gemm_store(dA, U, dW2, N, d, M, true, true, nullptr, ws, s));
+  const int parts = cdiv(M, UNF_DG_ROWS);
+  CODA_TRY(launch_status(launch_ex(unf_dg_partial_kernel, dim3(cdiv(d, 256), parts), dim3(256), 0, s, 1,
+                                   (const __nv_bfloat16*)du, cbf(H), r, part, M, d)));
+  CODA_TRY(launch_status(launch_ex(col_reduce_kernel, dim3(cdiv(d, 256)), dim3(256), 0, s, 1, (const float*)part,
+                                   parts, d, dg)));
+  CODA_TRY(launch_status(launch_ex(unf_rmsnorm_bwd_kernel, dim3(M), dim3(UNF_THREADS), 0, s, 1,
+                                   (const __nv_bfloat16*)du, cbf(H), cbf(g), r, cbf(dH_in_or_null), bf(dR), d)));
+  CODA_TRY(gemm_store(dR, W1, dX, M, K, d, false, true, nullptr, ws, s));
+  CODA_TRY(gemm_store(dR, X, dW1, d, K, M, true, true, nullptr, ws, s));
   return CODA_OK;
 }
 
@@ -581,6 +753,7 @@ extern "C" coda_status coda_grg_fwd_prefolded_static(const void* X, const void* 
     if (!make_operand_map(&ta, X, M, K, false, BM) || !make_operand_map(&tb, W1, d, K, false, pair ? BN / 2 : BN))
       return CODA_ERR_CUDA;
     GemmParams p = base_params(M, d, K, BN, scratch, pair);
+    p.group_m = pick_group(M, d, K, p.num_m_tiles, p.num_n_tiles, pair, num_sms());
     p.out = bf(H);
     p.ldo = d;
     p.in0 = cbf(R);
@@ -589,7 +762,7 @@ extern "C" coda_status coda_grg_fwd_prefolded_static(const void* X, const void* 
     p.ld_part = T;
     CODA_TRY((launch_gemm<EPI_RESID_RMS, false, false>(ta, tb, p, s, pair)));
   }
-  rms_rowreduce_kernel<<<cdiv(M, 256), 256, 0, s>>>(P, T, r, M, 1.0f / (float)d, eps);
-  CODA_TRY(launch_status(cudaPeekAtLastError()));
+  CODA_TRY(launch_status(launch_ex(rms_rowreduce_kernel, dim3(cdiv(M, 256)), dim3(256), 0, s, 1, (const float*)P, T,
+                                   r, M, 1.0f / (float)d, eps)));
   return gemm_swiglu(H, W2g, r, Y, AB_or_null, M, d, F, scratch, s);
 }

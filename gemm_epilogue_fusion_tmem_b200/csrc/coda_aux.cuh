@@ -14,6 +14,7 @@ namespace coda {
 // the epilogue entirely).
 __global__ void fold_gain_kernel(const __nv_bfloat16* __restrict__ W2, const __nv_bfloat16* __restrict__ g,
                                  __nv_bfloat16* __restrict__ W2g, int d, long long n_vec8) {
+  griddep_wait();
   const long long stride = (long long)gridDim.x * blockDim.x;
   for (long long v = (long long)blockIdx.x * blockDim.x + threadIdx.x; v < n_vec8; v += stride) {
     const long long e = v * 8;
@@ -32,6 +33,7 @@ __global__ void fold_gain_kernel(const __nv_bfloat16* __restrict__ W2, const __n
 // (kucoin.com (ru) CODA article, «В «Финале» спрятаны сокровища»).
 __global__ void rms_rowreduce_kernel(const float* __restrict__ P, int T, float* __restrict__ r, int M,
                                      float inv_d, float eps) {
+  griddep_wait();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= M) return;
   const float* row = P + (size_t)i * T;
@@ -70,6 +72,7 @@ __global__ void __launch_bounds__(ROWSTAT_THREADS)
                               const float* __restrict__ r, __nv_bfloat16* __restrict__ dAp,
                               float* __restrict__ c, int F, float inv_d) {
   __shared__ float scratch[32];
+  griddep_wait();
   const int row = blockIdx.x;
   const __nv_bfloat16* dy = dY + (size_t)row * F;
   const __nv_bfloat16* a = AB + (size_t)row * 2 * F;
@@ -102,6 +105,7 @@ __global__ void __launch_bounds__(ROWSTAT_THREADS)
 
 // dg_j = sum_t Pg[t, j]: reduce the dn GEMM's per-32-row column partials.
 __global__ void col_reduce_kernel(const float* __restrict__ Pg, int rows, int d, float* __restrict__ dg) {
+  griddep_wait();
   const int j = blockIdx.x * blockDim.x + threadIdx.x;
   if (j >= d) return;
   float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;

@@ -31,7 +31,6 @@ constexpr int UMMA_K = 16;
 constexpr int MN_CHUNK_BYTES = 64 * BK * 2;  // one [64 k][64 mn] MN-major chunk, 8 KiB
 constexpr int NUM_THREADS = 192;
 constexpr uint32_t TMEM_COLS = 2 * BN;
-constexpr int GROUP_M = 16;          // tile rasterisation: 16 row tiles per group
 
 enum Epi : int {
   EPI_STORE = 0,       // out = bf16(acc [* g_col])
@@ -48,6 +47,7 @@ struct GemmParams {
   int num_m_tiles;
   int num_n_tiles;
   int k_blocks;
+  int group_m;      // rasterisation (see tile_coords): >0 row-tile groups, <0 column-tile groups
   int split;        // EPI_SWIGLU: row offset of the up half in B and column offset of b in AB;
                     // EPI_SWIGLU_BWD: column offset of b / db (= F)
   __nv_bfloat16* out;
@@ -66,14 +66,29 @@ struct GemmParams {
   uint32_t kernel_id;
 };
 
-__device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int& m_blk, int& n_blk) {
-  const int group_size = GROUP_M * num_n;
-  const int group = tile / group_size;
-  const int first_m = group * GROUP_M;
-  const int gm = min(num_m - first_m, GROUP_M);
-  const int local = tile - group * group_size;
-  m_blk = first_m + local % gm;
-  n_blk = local / gm;
+// Tile order.  group > 0: groups of `group` row tiles, the row tile varying
+// fastest inside a group, so the group's A rows stay in L2 while B streams
+// through.  group < 0: the same with the roles of rows and columns swapped
+// (groups of -group column tiles, column tile fastest).
+__device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int group, int& m_blk, int& n_blk) {
+  if (group > 0) {
+    const int group_size = group * num_n;
+    const int g = tile / group_size;
+    const int first_m = g * group;
+    const int gm = min(num_m - first_m, group);
+    const int local = tile - g * group_size;
+    m_blk = first_m + local % gm;
+    n_blk = local / gm;
+  } else {
+    const int gsz = -group;
+    const int group_size = gsz * num_m;
+    const int g = tile / group_size;
+    const int first_n = g * gsz;
+    const int gn = min(num_n - first_n, gsz);
+    const int local = tile - g * group_size;
+    n_blk = first_n + local % gn;
+    m_blk = local / gn;
+  }
 }
 
 // Load 32 bf16 starting at p (16-byte aligned) as floats; zeros when !valid.
@@ -311,6 +326,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if constexpr (PAIR) cluster_sync(); else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // The set-up above overlaps the previous kernel's tail; global memory is
+  // touched only after it has completed.  The next kernel may start its own
+  // set-up as soon as SMs free up.
+  griddep_wait();
+  griddep_launch_dependents();
 
   const WaitCtl ctl{abort_flag, p.status, p.wait_limit_ns, p.kernel_id};
   const int num_tiles = p.num_m_tiles * p.num_n_tiles;
@@ -325,7 +345,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool ok = true;
       for (int tile = first_tile; tile < num_tiles && ok; tile += tile_step) {
         int m_blk, n_blk;
-        tile_coords(tile, p.num_m_tiles, p.num_n_tiles, m_blk, n_blk);
+        tile_coords(tile, p.num_m_tiles, p.num_n_tiles, p.group_m, m_blk, n_blk);
         const int a_row = m_blk * C::TILE_M + (int)rank * 128;
         for (int kb = 0; kb < p.k_blocks; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, ctl, 0, kWaitEmpty)) {
@@ -449,7 +469,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t acc_phase = 0;
     for (int tile = first_tile; tile < num_tiles; tile += tile_step) {
       int m_blk, n_blk;
-      tile_coords(tile, p.num_m_tiles, p.num_n_tiles, m_blk, n_blk);
+      tile_coords(tile, p.num_m_tiles, p.num_n_tiles, p.group_m, m_blk, n_blk);
       // Warp-uniform outcome: tcgen05.ld below needs all 32 lanes converged.
       const bool ok = mbar_wait(&tfull[acc], acc_phase, ctl, 2 + q, kWaitAccFull);
       if (!__all_sync(0xffffffffu, ok)) break;

@@ -197,6 +197,38 @@ coda_status coda_swiglu_bwd(const void* dOut, const void* X, const void* Wgu, co
                             void* dX, void* dWgu, void* dWdown,
                             int M, int d, int F, void* ws, size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------- unfused comparison sequence */
+
+/* The same block run operator by operator, the way a framework without
+ * epilogue fusion runs it (the operator boundaries that the pages identify as
+ * the source of the memory traffic: toolin.ai §課題; kucoin (ru) «Налог на
+ * лень»).  Every intermediate goes to HBM and back; the GEMMs are this
+ * library's plain-store tcgen05 GEMMs, so comparing these calls with
+ * coda_grg_fwd / coda_grg_bwd isolates what the fusion saves.  For
+ * measurement and error comparison; results agree with the fused path to
+ * bf16 storage precision.
+ *
+ * Forward: T = X W1^T;  H = T + R;  r, U = bf16(RMSNorm(H) * g);
+ *          AB = U W2^T (the pre-activations [a | b]);  Y = silu(a) * b.
+ * Outputs as coda_grg_fwd plus U [M, d] bf16 (the normalised activations an
+ * unfused backward keeps).  AB is required.
+ * Backward: dA = SwiGLU'(dY, AB);  du = dA W2;  dW2 = dA^T U;
+ *          dg_j = sum_i du_ij H_ij r_i;  dR = dH = RMSNorm'(du, H, g, r) (+dH_in);
+ *          dX = dH W1;  dW1 = dH^T X.
+ * Shape rules as coda_grg_fwd.  Workspaces from the *_workspace_bytes calls. */
+size_t coda_grg_fwd_unfused_workspace_bytes(int M, int K, int d, int N);
+coda_status coda_grg_fwd_unfused(const void* X, const void* W1, const void* R, const void* g, const void* W2,
+                                 void* H, float* r, void* Y, void* AB, void* U,
+                                 int M, int K, int d, int N, float eps,
+                                 void* ws, size_t ws_bytes, void* stream);
+size_t coda_grg_bwd_unfused_workspace_bytes(int M, int K, int d, int N);
+coda_status coda_grg_bwd_unfused(const void* dY, const void* dH_in_or_null,
+                                 const void* X, const void* W1, const void* H, const float* r,
+                                 const void* AB, const void* U, const void* g, const void* W2,
+                                 void* dX, void* dR, void* dW1, void* dW2, float* dg,
+                                 int M, int K, int d, int N,
+                                 void* ws, size_t ws_bytes, void* stream);
+
 /* ---------------------------------------------------------------- forward without any allocation */
 
 /* Upper bound on M * ceil(d / 256) for coda_grg_fwd_prefolded_static: the

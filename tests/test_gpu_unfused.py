@@ -1,0 +1,59 @@
+"""The unfused comparison sequence, and the fused path's error against it.
+
+The unfused calls run the block operator by operator (every intermediate in
+HBM).  They are checked against the pure fp64 oracle within the bound derived
+from bf16 storage, and the fused path's error must be comparable or smaller:
+the pages report the reparameterisation's numerical error as comparable to the
+PyTorch reference and sometimes smaller, thanks to the mainloop's fp32
+accumulator (kucoin.com (ru) CODA article, section «Результаты эксперимента»).
+The comparison is rms error against the pure fp64 oracle, fused <= 1.5x
+unfused (the factor is a chosen allowance, not a figure from the pages).
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from gemm_epilogue_fusion_tmem_b200 import synth
+from oracle import coda_oracle as O
+from tests.parity import assert_pure, f64
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    (256, 512, 512, 1024, 1e-6),
+    (200, 320, 384, 320, 1e-5),
+    (2048, 1024, 1024, 2816, 1e-6),
+]
+
+
+def _rms_err(gpu, ref):
+    g = f64(gpu)
+    return float(np.sqrt(np.mean((g - ref) ** 2)))
+
+
+@pytest.mark.parametrize("M,K,d,F,eps", CASES)
+def test_unfused_matches_oracle_and_fused_error_is_comparable(cuda_lib, M, K, d, F, eps):
+    t = synth.grg_inputs(M, K, d, F, seed=21, dH_in=True)
+    td = {k: v.cuda() for k, v in t.items()}
+    fu = cuda_lib.grg_fwd(td["X"], td["W1"], td["R"], td["g"], td["W2"], eps)
+    bu = cuda_lib.grg_bwd(td["dY"], td["X"], td["W1"], fu["H"], fu["r"], fu["AB"], td["g"], td["W2"],
+                          dH_in=td["dH_in"])
+    uf = cuda_lib.grg_fwd_unfused(td["X"], td["W1"], td["R"], td["g"], td["W2"], eps)
+    ub = cuda_lib.grg_bwd_unfused(td["dY"], td["X"], td["W1"], uf["H"], uf["r"], uf["AB"], uf["U"], td["g"],
+                                  td["W2"], dH_in=td["dH_in"])
+    torch.cuda.synchronize()
+    X, W1, R, g, W2, dY, dH_in = (f64(t[k]) for k in ("X", "W1", "R", "g", "W2", "dY", "dH_in"))
+    fwd = O.grg_forward(X, W1, R, g, W2, eps)
+    bwd = O.grg_backward(dY, X, W1, R, g, W2, eps, dH_in=dH_in, fwd=fwd)
+    tag = f"M={M} K={K} d={d} F={F}"
+    unf = {"H": uf["H"], "Y": uf["Y"], "a": uf["AB"][:, :F], "b": uf["AB"][:, F:], **ub}
+    fus = {"H": fu["H"], "Y": fu["Y"], "a": fu["AB"][:, :F], "b": fu["AB"][:, F:], **bu}
+    ref = {**{k: fwd[k] for k in ("H", "Y", "a", "b")}, **{k: bwd[k] for k in ("dX", "dR", "dW1", "dW2", "dg")}}
+    for k, v in unf.items():
+        assert_pure(v, ref[k], f"unfused {tag} {k}")
+    np.testing.assert_allclose(f64(uf["r"]), fwd["r"], rtol=1e-3)
+    for k in ref:
+        e_f, e_u = _rms_err(fus[k], ref[k]), _rms_err(unf[k], ref[k])
+        rms = float(np.sqrt(np.mean(ref[k] ** 2)))
+        assert e_f <= 1.5 * e_u + 1e-4 * rms, f"{tag} {k}: fused rms error {e_f:.3g} vs unfused {e_u:.3g}"
