@@ -219,6 +219,31 @@ def _recorded_traffic(kernel: str, workload: str):
     return None
 
 
+# ----------------------------------------------------------------------------- ranks (replicas)
+
+def dist_env():
+    """(rank, world, local_rank) from the torchrun environment (1 process when absent)."""
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(x: float, device, world: int) -> float:
+    """The largest value of x over all ranks (every rank gets it)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(flops_per_step: float, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job TFLOP/s: every rank runs its own replica of the workload, the
+    job's time is the slowest rank's (weak scaling, no data-path collective)."""
+    return flops_per_step * steps * world / (max_ms / 1e3) / 1e12
+
+
 # ----------------------------------------------------------------------------- the CUDA arm
 
 def _setup(kind, s, bwd, device):
@@ -335,9 +360,7 @@ def run_coda(a):
     import torch
     import torch.distributed as dist
     kind, s, bwd = WORKLOADS[a.workload]
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, world, local = dist_env()
     if not torch.cuda.is_available():
         raise SystemExit("bench.py: no CUDA device (the library has no CPU path)")
     torch.cuda.set_device(local)
@@ -372,11 +395,40 @@ def run_coda(a):
     status, detail = ws.query()
     if status != 0:
         raise SystemExit(f"bench.py: device status {status} detail {detail:#x}")
-    t = torch.tensor([ms_total], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
-    value = flops * a.steps * world / (ms_max / 1e3) / 1e12
+    ms_max = max_over_ranks(ms_total, device, world)
+    value = replica_throughput(flops, a.steps, world, ms_max)
+
+    # The activation-side gain variant (Hg from GEMM1's epilogue, no gain fold).
+    variants = {}
+    if kind == "grg":
+        from gemm_epilogue_fusion_tmem_b200 import binding as B
+        lib = B.library()
+        hws = B.Workspace(max(lib.coda_grg_fwd_hg_workspace_bytes(s["M"], s["K"], s["d"], 2 * s["F"], 0),
+                              lib.coda_grg_bwd_workspace_bytes(s["M"], s["K"], s["d"], 2 * s["F"])), device)
+        hf = {k: outs[k] for k in ("H", "r", "Y", "AB")}
+        hb = {k: outs[k] for k in ("dX", "dR", "dW1", "dW2", "dg")} if bwd else {}
+
+        def hstep():
+            B.grg_fwd_hg(dev["X"], dev["W1"], dev["R"], dev["g"], dev["W2"], s["eps"], out=hf, ws=hws)
+            if bwd:
+                B.grg_bwd(dev["dY"], dev["X"], dev["W1"], hf["H"], hf["r"], hf["AB"], dev["g"], dev["W2"], out=hb,
+                          ws=hws)
+
+        for _ in range(max(a.warmup, 3)):
+            hstep()
+        torch.cuda.synchronize()
+        barrier()
+        e0.record(st)
+        for _ in range(a.steps):
+            hstep()
+        e1.record(st)
+        torch.cuda.synchronize()
+        barrier()
+        h_ms = max_over_ranks(e0.elapsed_time(e1), device, world)
+        variants["activation_gain"] = {"ms_per_step": round(h_ms / a.steps, 4),
+                                       "value": round(replica_throughput(flops, a.steps, world, h_ms), 2),
+                                       "what": "coda_grg_fwd_hg: GEMM1 stores H*g, GEMM2 reads W2 unfolded"}
+        del hws
 
     # The unfused comparison sequence, timed the same way right after.
     unfused = None
@@ -392,12 +444,9 @@ def run_coda(a):
         e1.record(st)
         torch.cuda.synchronize()
         barrier()
-        tu = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=device)
-        if world > 1:
-            dist.all_reduce(tu, op=dist.ReduceOp.MAX)
-        u_ms = float(tu.item())
+        u_ms = max_over_ranks(e0.elapsed_time(e1), device, world)
         unfused = {"ms_per_step": round(u_ms / a.steps, 4),
-                   "value": round(flops * a.steps * world / (u_ms / 1e3) / 1e12, 2), "unit": "TFLOP/s",
+                   "value": round(replica_throughput(flops, a.steps, world, u_ms), 2), "unit": "TFLOP/s",
                    "fused_speedup": round(u_ms / ms_max, 4), "gpu_launches_per_step": ulaunch,
                    "what": "same GEMM kernels with plain stores; residual add, RMSNorm, SwiGLU and their backward "
                            "as separate HBM-round-trip kernels"}
@@ -439,10 +488,8 @@ def run_coda(a):
         e1.record(st)
         torch.cuda.synchronize()
         barrier()
-        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=device)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e = {"value": round(flops * n_e2e * world / (float(te.item()) / 1e3) / 1e12, 2), "unit": "TFLOP/s",
+        te = max_over_ranks(e0.elapsed_time(e1), device, world)
+        e2e = {"value": round(replica_throughput(flops, n_e2e, world, te), 2), "unit": "TFLOP/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": n_e2e}
 
     cpu = None
@@ -470,6 +517,7 @@ def run_coda(a):
             "roofline": roofline,
             "cpu_baseline": cpu,
             "unfused": unfused,
+            "variants": variants or None,
             "e2e": e2e,
             "gpu_launches": launches * a.steps,
             "clocks": clk.summary(),
@@ -480,11 +528,11 @@ def run_coda(a):
 
 
 def run_reference(a):
-    """The reference arm: the fp64 CPU oracle on the host cores, bounded samples of the workload."""
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
+    """The reference arm: the fp64 CPU oracle on the host cores, bounded samples of the workload.
+    Under torchrun only rank 0 runs it; the other ranks return without work."""
+    rank, world, _ = dist_env()
     if rank != 0:
-        return
+        return None
     kind, s, bwd = WORKLOADS[a.workload]
     inputs = _oracle_inputs(kind, s)
     probe = min(64, s["M"])
@@ -513,6 +561,7 @@ def run_reference(a):
         "e2e": {"value": round(value, 4), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+    return line
 
 
 def main():

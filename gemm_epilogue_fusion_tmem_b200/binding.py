@@ -67,6 +67,8 @@ def library() -> ctypes.CDLL:
             "coda_swiglu_fwd": (I, [P, P, P, P, P, P, I, I, I, P, S, P]),
             "coda_swiglu_bwd_workspace_bytes": (S, [I, I, I]),
             "coda_swiglu_bwd": (I, [P, P, P, P, P, P, P, P, P, I, I, I, P, S, P]),
+            "coda_grg_fwd_hg_workspace_bytes": (S, [I, I, I, I, I]),
+            "coda_grg_fwd_hg": (I, [P] * 10 + [I, I, I, I, F, P, S, P]),
             "coda_grg_fwd_unfused_workspace_bytes": (S, [I, I, I, I]),
             "coda_grg_fwd_unfused": (I, [P] * 10 + [I, I, I, I, F, P, S, P]),
             "coda_grg_bwd_unfused_workspace_bytes": (S, [I, I, I, I]),
@@ -235,6 +237,35 @@ def grg_fwd(X, W1, R, g, W2, eps: float, W2g=None, save_ab: bool = True, out: di
     _check(lib.coda_grg_fwd(_ptr(X), _ptr(W1), _ptr(R), _ptr(g), _ptr(W2), _ptr(W2g), _ptr(o["H"]),
                             _ptr(o["r"]), _ptr(o["Y"]), _ptr(AB), M, K, d, N, float(eps),
                             ws.ptr(), ws.nbytes, _stream()), "coda_grg_fwd")
+    return o
+
+
+def grg_fwd_hg(X, W1, R, g, W2, eps: float, save_ab: bool = True, keep_hg: bool = False, out: dict | None = None,
+               ws: Workspace | None = None) -> dict:
+    """Forward with the gain on the activation side (Hg = H*g from GEMM1's epilogue); returns H, r, Y, AB (, Hg)."""
+    lib = library()
+    M, K = X.shape
+    d = W1.shape[0]
+    N = W2.shape[0]
+    F = N // 2
+    _req(X, "X"), _req(W1, "W1", shape=(d, K)), _req(R, "R", shape=(M, d))
+    _req(g, "g", shape=(d,)), _req(W2, "W2", shape=(N, d))
+    o = dict(out or {})
+    dev = X.device
+    want = [("H", (M, d), torch.bfloat16), ("r", (M,), torch.float32), ("Y", (M, F), torch.bfloat16)]
+    if save_ab:
+        want.append(("AB", (M, N), torch.bfloat16))
+    if keep_hg:
+        want.append(("Hg", (M, d), torch.bfloat16))
+    for k, shape, dt in want:
+        if k not in o:
+            o[k] = torch.empty(*shape, dtype=dt, device=dev)
+        _req(o[k], k, dt, shape)
+    Hg = o.get("Hg") if keep_hg else None
+    ws = ws or workspace(lib.coda_grg_fwd_hg_workspace_bytes(M, K, d, N, int(Hg is not None)), dev)
+    _check(lib.coda_grg_fwd_hg(_ptr(X), _ptr(W1), _ptr(R), _ptr(g), _ptr(W2), _ptr(o["H"]), _ptr(Hg), _ptr(o["r"]),
+                               _ptr(o["Y"]), _ptr(o.get("AB") if save_ab else None), M, K, d, N, float(eps),
+                               ws.ptr(), ws.nbytes, _stream()), "coda_grg_fwd_hg")
     return o
 
 

@@ -458,6 +458,55 @@ coda_status coda_grg_fwd(const void* X, const void* W1, const void* R, const voi
   return CODA_OK;
 }
 
+size_t coda_grg_fwd_hg_workspace_bytes(int M, int K, int d, int N, int hg_given) {
+  (void)K, (void)N;
+  if (M < 1 || d < 1) return kStatusBytes;
+  const int T = cdiv(d, kRmsTile);
+  size_t tot = align_up(kStatusBytes + (size_t)M * T * 4, 256);
+  if (!hg_given) tot += align_up((size_t)M * d * 2, 256);
+  return tot;
+}
+
+coda_status coda_grg_fwd_hg(const void* X, const void* W1, const void* R, const void* g, const void* W2, void* H,
+                            void* Hg_or_null, float* r, void* Y, void* AB_or_null, int M, int K, int d, int N,
+                            float eps, void* ws, size_t ws_bytes, void* stream) {
+  if (!X || !W1 || !R || !g || !W2 || !H || !r || !Y || !ws) return CODA_ERR_INVALID_ARG;
+  if (!(eps > 0.f)) return CODA_ERR_INVALID_ARG;
+  CODA_TRY(check_grg_shapes(M, K, d, N));
+  const void* ptrs[] = {X, W1, R, g, W2, H, Hg_or_null, r, Y, AB_or_null, ws};
+  for (const void* q : ptrs)
+    if (q && !aligned16(q)) return CODA_ERR_MISALIGNED;
+  if (ws_bytes < coda_grg_fwd_hg_workspace_bytes(M, K, d, N, Hg_or_null != nullptr)) return CODA_ERR_WORKSPACE_TOO_SMALL;
+  int dev;
+  CODA_TRY(current_device(dev));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  float* P = reinterpret_cast<float*>(wsb + kStatusBytes);
+  const int T = cdiv(d, kRmsTile);
+  void* Hg = Hg_or_null ? Hg_or_null : wsb + align_up(kStatusBytes + (size_t)M * T * 4, 256);
+  const int F = N / 2;
+  {
+    const bool pair = use_pair();
+    CUtensorMap ta, tb;
+    if (!make_operand_map(&ta, X, M, K, false, BM) || !make_operand_map(&tb, W1, d, K, false, pair ? BN / 2 : BN))
+      return CODA_ERR_CUDA;
+    GemmParams p = base_params(M, d, K, BN, ws, pair);
+    p.group_m = pick_group(M, d, K, p.num_m_tiles, p.num_n_tiles, pair, num_sms());
+    p.out = bf(H);
+    p.ldo = d;
+    p.in0 = cbf(R);
+    p.ld_in0 = d;
+    p.part = P;
+    p.ld_part = T;
+    p.out2 = bf(Hg);
+    p.colvec = cbf(g);
+    CODA_TRY((launch_gemm<EPI_RESID_RMS, false, false>(ta, tb, p, s, pair)));
+  }
+  CODA_TRY(launch_status(launch_ex(rms_rowreduce_kernel, dim3(cdiv(M, 256)), dim3(256), 0, s, 1, (const float*)P, T,
+                                   r, M, 1.0f / (float)d, eps)));
+  return gemm_swiglu(Hg, W2, r, Y, AB_or_null, M, d, F, ws, s);
+}
+
 // ------------------------------------------------------------------ GRG backward
 
 namespace {
@@ -526,7 +575,7 @@ coda_status coda_grg_bwd(const void* dY, const void* dH_in_or_null, const void* 
     CODA_TRY((launch_gemm<EPI_DN, false, true>(ta, tb, p, s, pair)));
   }
   // One partial row per 32 output rows of every (possibly partial) row tile.
-  CODA_TRY(launch_status(launch_ex(col_reduce_kernel, dim3(cdiv(d, 256)), dim3(256), 0, s, 1, (const float*)Pg,
+  CODA_TRY(launch_status(launch_ex(col_reduce_kernel, dim3(cdiv(d, 32)), dim3(COLRED_THREADS), 0, s, 1, (const float*)Pg,
                                    cdiv(M, tile_m(pair)) * tile_m(pair) / 32, d, dg)));
   // dW2 = g * (dA'^T H).
   CODA_TRY(gemm_store(dAp, H, dW2, N, d, M, true, true, g, ws, s));
@@ -688,7 +737,7 @@ coda_status coda_grg_bwd_unfused(const void* dY, const void* dH_in_or_null, cons
   const int parts = cdiv(M, UNF_DG_ROWS);
   CODA_TRY(launch_status(launch_ex(unf_dg_partial_kernel, dim3(cdiv(d, 256), parts), dim3(256), 0, s, 1,
                                    (const __nv_bfloat16*)du, cbf(H), r, part, M, d)));
-  CODA_TRY(launch_status(launch_ex(col_reduce_kernel, dim3(cdiv(d, 256)), dim3(256), 0, s, 1, (const float*)part,
+  CODA_TRY(launch_status(launch_ex(col_reduce_kernel, dim3(cdiv(d, 32)), dim3(COLRED_THREADS), 0, s, 1, (const float*)part,
                                    parts, d, dg)));
   CODA_TRY(launch_status(launch_ex(unf_rmsnorm_bwd_kernel, dim3(M), dim3(UNF_THREADS), 0, s, 1,
                                    (const __nv_bfloat16*)du, cbf(H), cbf(g), r, cbf(dH_in_or_null), bf(dR), d)));

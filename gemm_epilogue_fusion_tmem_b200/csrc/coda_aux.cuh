@@ -104,20 +104,30 @@ __global__ void __launch_bounds__(ROWSTAT_THREADS)
 }
 
 // dg_j = sum_t Pg[t, j]: reduce the dn GEMM's per-32-row column partials.
-__global__ void col_reduce_kernel(const float* __restrict__ Pg, int rows, int d, float* __restrict__ dg) {
+// One block per 32 columns; warp w sums rows w, w+8, ... (lane = column, so
+// each warp load is one 128-byte line), then the 8 warp sums are added in a
+// fixed order, so the result is bit-reproducible.
+constexpr int COLRED_THREADS = 256;
+__global__ void __launch_bounds__(COLRED_THREADS)
+    col_reduce_kernel(const float* __restrict__ Pg, int rows, int d, float* __restrict__ dg) {
+  __shared__ float part[COLRED_THREADS / 32][32];
   griddep_wait();
-  const int j = blockIdx.x * blockDim.x + threadIdx.x;
-  if (j >= d) return;
-  float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-  int t = 0;
-  for (; t + 4 <= rows; t += 4) {
-    s0 += Pg[(size_t)t * d + j];
-    s1 += Pg[(size_t)(t + 1) * d + j];
-    s2 += Pg[(size_t)(t + 2) * d + j];
-    s3 += Pg[(size_t)(t + 3) * d + j];
+  const int lane = threadIdx.x & 31;
+  const int w = threadIdx.x >> 5;
+  const int j = blockIdx.x * 32 + lane;
+  float s = 0.f;
+  if (j < d) {
+#pragma unroll 4
+    for (int t = w; t < rows; t += COLRED_THREADS / 32) s += Pg[(size_t)t * d + j];
   }
-  for (; t < rows; ++t) s0 += Pg[(size_t)t * d + j];
-  dg[j] = (s0 + s1) + (s2 + s3);
+  part[w][lane] = s;
+  __syncthreads();
+  if (w == 0 && j < d) {
+    float tot = 0.f;
+#pragma unroll
+    for (int k = 0; k < COLRED_THREADS / 32; ++k) tot += part[k][lane];
+    dg[j] = tot;
+  }
 }
 
 }  // namespace coda

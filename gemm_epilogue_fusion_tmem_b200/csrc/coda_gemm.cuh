@@ -34,7 +34,7 @@ constexpr uint32_t TMEM_COLS = 2 * BN;
 
 enum Epi : int {
   EPI_STORE = 0,       // out = bf16(acc [* g_col])
-  EPI_RESID_RMS = 1,   // H = bf16(acc + R); P[row, ntile] = sum bf16(H)^2
+  EPI_RESID_RMS = 1,   // H = bf16(acc + R); P[row, ntile] = sum bf16(H)^2; optional Hg = bf16(H*g)
   EPI_SWIGLU = 2,      // a = r*acc_gate, b = r*acc_up; Y = silu(a)*b; AB = [a|b]
   EPI_DN = 3,          // dH = g*acc - c*H (+dH_in); column partials of acc*H
   EPI_SWIGLU_BWD = 4,  // dY = acc; da, db from a, b; dA = [da|db]
@@ -59,7 +59,7 @@ struct GemmParams {
   const float* rowvec;          // r (SWIGLU, optional), c (DN)
   float* part;                  // P (RESID_RMS), Pg (DN)
   int ld_part;
-  __nv_bfloat16* out2;          // AB (SWIGLU), optional
+  __nv_bfloat16* out2;          // AB (SWIGLU), Hg (RESID_RMS), optional
   int ldo2;
   uint32_t* status;
   unsigned long long wait_limit_ns;
@@ -174,6 +174,14 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbas
         __nv_bfloat16* dst = p.out + (size_t)row * p.ldo + n0 + c;
 #pragma unroll
         for (int j = 0; j < 4; ++j) stg_v4(dst + 8 * j, hq[j]);
+      }
+      if (p.out2 != nullptr) {
+        // Activation-side gain: Hg = bf16(H * g), the second GEMM's operand.
+        float g[32];
+        load32_bf16(p.colvec + n0 + c, true, g);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) g[i] *= v[i] + rres[i];
+        if (rv) store32_bf16(p.out2 + (size_t)row * p.ldo + n0 + c, g);
       }
     }
     if (rv) p.part[(size_t)row * p.ld_part + n_blk] = ss;

@@ -139,6 +139,25 @@ coda_status coda_grg_fwd(const void* X, const void* W1, const void* R, const voi
                          int M, int K, int d, int N, float eps,
                          void* ws, size_t ws_bytes, void* stream);
 
+/* Workspace for coda_grg_fwd_hg: status word, P, and Hg [M, d] bf16 when the
+ * caller passes no Hg buffer. */
+size_t coda_grg_fwd_hg_workspace_bytes(int M, int K, int d, int N, int hg_given);
+
+/* The same forward with the RMSNorm gain applied on the activation side
+ * instead of being folded into W2: GEMM1's epilogue also stores
+ * Hg = bf16(H * g) (the elementwise-transform and tile-store primitives of
+ * the five-primitive table), and GEMM2 reads Hg with the unmodified W2:
+ *   acc = Hg W2^T;  a = r_i acc_gate, b = r_i acc_up;  Y = silu(a) * b.
+ * diag(r) (H diag(g)) W2^T equals the folded form exactly, so the results are
+ * the forward's up to bf16 rounding; the 4*N*d bytes of the gain fold are
+ * replaced by M*d*2 bytes of Hg.  Hg_or_null: optional output [M, d] bf16
+ * (placed in the workspace when null).  Other arguments and the shape rules
+ * as coda_grg_fwd; the backward is coda_grg_bwd unchanged. */
+coda_status coda_grg_fwd_hg(const void* X, const void* W1, const void* R, const void* g, const void* W2,
+                            void* H, void* Hg_or_null, float* r, void* Y, void* AB_or_null,
+                            int M, int K, int d, int N, float eps,
+                            void* ws, size_t ws_bytes, void* stream);
+
 /* ---------------------------------------------------------------- GRG backward */
 
 /* Workspace for coda_grg_bwd: status word, dA' [M, N] bf16, c [M] fp32 and

@@ -242,23 +242,29 @@ def _ident(x):
     return x
 
 
-def grg_forward_stored(X, W1, R, g, W2, eps: float, store=round_bf16) -> dict:
+def grg_forward_stored(X, W1, R, g, W2, eps: float, store=round_bf16, gain: str = "weight") -> dict:
     """grg_forward with the method's dataflow at storage precision.
 
       H   = store(X W1^T + R)                  stored by GEMM1, read by the rest
       r   = 1/sqrt(mean_j H_ij^2 + eps)        from the stored H
-      W2g = store(W2 diag(g))                  the gain folded into GEMM2's weight
-      A   = diag(r) (H W2g^T)                  r deferred past GEMM2 (the pages' identity)
+      gain = "weight":     W2g = store(W2 diag(g)),  A = diag(r) (H W2g^T)
+      gain = "activation": Hg = store((X W1^T + R) diag(g)), A = diag(r) (Hg W2^T)
+                                               r deferred past GEMM2 (the pages' identity)
       a, b = A[:, :F], A[:, F:];  Y = silu(a) * b   (Y from the unrounded a, b)
       a_s, b_s = store(a), store(b)            saved for the backward
     """
     X, W1, R, g, W2 = map(_f64, (X, W1, R, g, W2))
-    H = store(X @ W1.T + R)
+    H_exact = X @ W1.T + R
+    H = store(H_exact)
     d = H.shape[1]
     ms = np.sum(H * H, axis=1) / d
     r = 1.0 / np.sqrt(ms + eps)
-    W2g = store(W2 * g[None, :])
-    A = r[:, None] * (H @ W2g.T)
+    if gain == "weight":
+        A = r[:, None] * (H @ store(W2 * g[None, :]).T)
+    elif gain == "activation":
+        A = r[:, None] * (store(H_exact * g[None, :]) @ W2.T)
+    else:
+        raise ValueError(f"gain must be 'weight' or 'activation', got {gain!r}")
     F = W2.shape[0] // 2
     a, b = A[:, :F], A[:, F:]
     Y = silu(a) * b

@@ -58,6 +58,21 @@ def test_grg_full_size(cuda_lib, name, M, K, d, F, eps, bwd, also_pure):
                 assert_pure(gb[k], b0[k], f"{name} {k}")
 
 
+def test_grg_full_size_activation_gain(cuda_lib):
+    """The 7B forward with Hg = bf16(H*g) from GEMM1 feeding GEMM2 (no gain fold)."""
+    M, K, d, F, eps = 8192, 4096, 4096, 11008, 1e-6
+    t = synth.grg_inputs(M, K, d, F, seed=0)
+    td = {k: v.cuda() for k, v in t.items()}
+    o = cuda_lib.grg_fwd_hg(td["X"], td["W1"], td["R"], td["g"], td["W2"], eps)
+    torch.cuda.synchronize()
+    gpu = {"H": f64(o["H"]), "Y": f64(o["Y"]), "a": f64(o["AB"][:, :F]), "b": f64(o["AB"][:, F:])}
+    del o, td
+    X, W1, R, g, W2 = (f64(t[k]) for k in ("X", "W1", "R", "g", "W2"))
+    fs = O.grg_forward_stored(X, W1, R, g, W2, eps, gain="activation")
+    for k, v in gpu.items():
+        assert_tol(v, fs[k], f"7B hg {k}")
+
+
 def test_grg_full_size_r(cuda_lib):
     """The fp32 row scale r of the 7B forward within 1e-3 relative of both oracles."""
     M, K, d, F, eps = 8192, 4096, 4096, 11008, 1e-6

@@ -200,3 +200,24 @@ def test_status_word_stays_clear(cuda_lib):
     ws = cuda_lib.workspace(1 << 20)
     st, detail = ws.query()
     assert st == 0 and detail == 0, f"device status {st} detail {detail:#x}"
+
+
+# ----------------------------------------------------------------------------- gain on the activation side
+
+@pytest.mark.parametrize("M,K,d,F,eps", GRG_CASES)
+def test_grg_forward_activation_gain(cuda_lib, M, K, d, F, eps):
+    """coda_grg_fwd_hg: Hg = bf16(H*g) from GEMM1's epilogue feeds GEMM2 with the unmodified W2."""
+    t = synth.grg_inputs(M, K, d, F, seed=7)
+    td = _cuda(t)
+    o = cuda_lib.grg_fwd_hg(td["X"], td["W1"], td["R"], td["g"], td["W2"], eps, keep_hg=True)
+    b = cuda_lib.grg_bwd(td["dY"], td["X"], td["W1"], o["H"], o["r"], o["AB"], td["g"], td["W2"])
+    torch.cuda.synchronize()
+    X, W1, R, g, W2, dY = (f64(t[k]) for k in ("X", "W1", "R", "g", "W2", "dY"))
+    fwd = O.grg_forward(X, W1, R, g, W2, eps)
+    fs = O.grg_forward_stored(X, W1, R, g, W2, eps, gain="activation")
+    tag = f"grg_fwd_hg M={M} K={K} d={d} F={F}"
+    _check_fwd(o, fwd, fs, tag)
+    assert_tol(o["Hg"], O.round_bf16(fwd["H"] * g[None, :]), f"{tag} Hg")
+    bs = O.grg_backward_stored(dY, X, W1, R, g, W2, eps, fwd=fs)
+    for k in ("dX", "dR", "dW1", "dW2", "dg"):
+        assert_tol(b[k], bs[k], f"{tag} bwd {k}", outlier_frac=BWD_OUTLIER_FRAC)

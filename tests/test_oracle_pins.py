@@ -330,9 +330,12 @@ def test_stored_functions_reduce_to_textbook_without_rounding():
     g = 1 + 0.1 * rng.standard_normal(d)
     dY, dH_in = rng.standard_normal((M, F)), rng.standard_normal((M, d))
     f0 = O.grg_forward(X, W1, R, g, W2, eps)
-    f1 = O.grg_forward_stored(X, W1, R, g, W2, eps, store=_ident)
-    for k in ("H", "r", "a", "b", "Y"):
-        np.testing.assert_allclose(f1[k], f0[k], rtol=1e-12, atol=1e-12, err_msg=k)
+    for gain in ("weight", "activation"):
+        f1 = O.grg_forward_stored(X, W1, R, g, W2, eps, store=_ident, gain=gain)
+        for k in ("H", "r", "a", "b", "Y"):
+            np.testing.assert_allclose(f1[k], f0[k], rtol=1e-12, atol=1e-12, err_msg=f"{gain} {k}")
+    with pytest.raises(ValueError):
+        O.grg_forward_stored(X, W1, R, g, W2, eps, gain="neither")
     b0 = O.grg_backward(dY, X, W1, R, g, W2, eps, dH_in=dH_in)
     b1 = O.grg_backward_stored(dY, X, W1, R, g, W2, eps, dH_in=dH_in, store=_ident)
     for k in ("dX", "dR", "dW1", "dW2", "dg"):
