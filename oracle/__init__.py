@@ -13,4 +13,6 @@ from .coda_oracle import (  # noqa: F401
     silu,
     swiglu_backward,
     swiglu_forward,
+    xent_backward,
+    xent_forward,
 )

@@ -55,6 +55,8 @@ __all__ = [
     "grg_backward_stored",
     "swiglu_forward_stored",
     "swiglu_backward_stored",
+    "xent_forward",
+    "xent_backward",
 ]
 
 
@@ -321,3 +323,44 @@ def swiglu_backward_stored(dOut, X, Wgu, Wdown, store=round_bf16, fwd: dict | No
     da, db = _swiglu_grads(dY, fwd["a_s"], fwd["b_s"])
     dA = store(np.concatenate([da, db], axis=1))
     return {"dY": dY, "dA": dA, "dWdown": dOut.T @ fwd["Y_s"], "dWgu": dA.T @ X, "dX": dA @ Wgu}
+
+
+# ----------------------------------------------------------------------------- cross-entropy
+
+def xent_forward(X, W, targets) -> dict:
+    """Cross-entropy of the LM-head GEMM, textbook order.
+
+      logits = X W^T              (X [M, d], W [V, d])
+      lse_i  = log sum_j exp(logits_ij)          (max-shifted for range)
+      loss_i = lse_i - logits_i,t_i
+    The pages name cross-entropy among the operations rewritten as
+    GEMM-epilogue programs, via a tile-wise log-sum-exp and the online
+    max / sum-exp statistics (toolin.ai five-primitive table, rows "tile-wise
+    reduction" and "stateful transform"; kucoin (ru) «В «Финале» спрятаны
+    сокровища»).  The oracle is the plain definition, not the tiled form.
+    """
+    X, W = _f64(X), _f64(W)
+    t = np.asarray(targets, dtype=np.int64)
+    logits = X @ W.T
+    m = np.max(logits, axis=1)
+    lse = m + np.log(np.sum(np.exp(logits - m[:, None]), axis=1))
+    loss = lse - logits[np.arange(X.shape[0]), t]
+    return {"logits": logits, "lse": lse, "loss": loss}
+
+
+def xent_backward(dloss, X, W, targets, fwd: dict | None = None, store=None) -> dict:
+    """Gradients of L = sum_i dloss_i loss_i (chain rule by hand):
+      dlogits_ij = dloss_i (softmax_ij - [j == t_i]);  dX = dlogits W;  dW = dlogits^T X.
+    store: optional rounding of dlogits where the method stores it (bf16)
+    before the two GEMMs read it; None keeps float64.
+    """
+    if fwd is None:
+        fwd = xent_forward(X, W, targets)
+    X, W, dloss = _f64(X), _f64(W), _f64(dloss)
+    t = np.asarray(targets, dtype=np.int64)
+    p = np.exp(fwd["logits"] - fwd["lse"][:, None])
+    p[np.arange(X.shape[0]), t] -= 1.0
+    dlogits = p * dloss[:, None]
+    if store is not None:
+        dlogits = store(dlogits)
+    return {"dlogits": dlogits, "dX": dlogits @ W, "dW": dlogits.T @ X}

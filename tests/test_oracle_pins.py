@@ -362,3 +362,52 @@ def test_stored_rounding_is_small_and_present():
     assert np.array_equal(f1["H"], O.round_bf16(f0["H"]))
     rel = np.sqrt(np.mean((f1["A"] - f0["A"]) ** 2)) / np.sqrt(np.mean(f0["A"] ** 2))
     assert 1e-4 < rel < 2 ** -8
+
+
+# ----------------------------------------------------------------------------- cross-entropy
+
+def test_xent_uniform_logits_closed_form():
+    """W = 0 gives equal logits: loss = log V for every target, softmax = 1/V."""
+    M, d, V = 5, 8, 37
+    X = np.random.default_rng(16).standard_normal((M, d))
+    W = np.zeros((V, d))
+    t = np.array([0, 3, 36, 10, 10])
+    f = O.xent_forward(X, W, t)
+    np.testing.assert_allclose(f["loss"], np.log(V), rtol=1e-15)
+    b = O.xent_backward(np.ones(M), X, W, t, fwd=f)
+    expect = np.full((M, V), 1.0 / V)
+    expect[np.arange(M), t] -= 1.0
+    np.testing.assert_allclose(b["dlogits"], expect, rtol=1e-14, atol=1e-16)
+
+
+def test_xent_matches_torch_cross_entropy_and_autograd():
+    torch.manual_seed(17)
+    M, d, V = 12, 16, 50
+    X = torch.randn(M, d, dtype=torch.float64, requires_grad=True)
+    W = (torch.randn(V, d, dtype=torch.float64) / 2).requires_grad_()
+    t = torch.randint(0, V, (M,))
+    dloss = torch.rand(M, dtype=torch.float64)
+    loss = Fn.cross_entropy(Fn.linear(X, W), t, reduction="none")
+    (loss * dloss).sum().backward()
+    f = O.xent_forward(X.detach().numpy(), W.detach().numpy(), t.numpy())
+    np.testing.assert_allclose(f["loss"], loss.detach().numpy(), rtol=1e-12)
+    b = O.xent_backward(dloss.numpy(), X.detach().numpy(), W.detach().numpy(), t.numpy(), fwd=f)
+    np.testing.assert_allclose(b["dX"], X.grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(b["dW"], W.grad.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_xent_shift_invariance_and_finite_differences():
+    """Adding a constant to a row's logits leaves the loss unchanged (a bias column
+    of X with a constant W column); the backward matches central differences."""
+    rng = np.random.default_rng(18)
+    M, d, V = 4, 6, 9
+    X, W = rng.standard_normal((M, d)), rng.standard_normal((V, d))
+    t = np.array([1, 8, 0, 4])
+    Xb = np.concatenate([X, np.ones((M, 1))], axis=1)
+    Wb = np.concatenate([W, np.full((V, 1), 5.0)], axis=1)
+    np.testing.assert_allclose(O.xent_forward(Xb, Wb, t)["loss"], O.xent_forward(X, W, t)["loss"], rtol=1e-12)
+    dloss = rng.standard_normal(M)
+    b = O.xent_backward(dloss, X, W, t)
+    p = {"X": X.copy(), "W": W.copy()}
+    _fd_check(lambda q: float(np.sum(dloss * O.xent_forward(q["X"], q["W"], t)["loss"])), p,
+              {"X": b["dX"], "W": b["dW"]}, ["X", "W"])
