@@ -38,6 +38,7 @@ WORKLOADS = {
     "7B": ("grg", dict(M=8192, K=4096, d=4096, F=11008, eps=1e-6), True),
     "70B": ("grg", dict(M=4096, K=8192, d=8192, F=28672, eps=1e-5), True),
     "swiglu": ("swiglu", dict(M=16384, d=4096, F=14336), True),
+    "xent": ("xent", dict(M=8192, d=4096, V=128256), True),
 }
 
 
@@ -63,6 +64,8 @@ def _peaks():
 
 
 def _flops(kind, s, bwd):
+    if kind == "xent":  # logits GEMM forward, dX and dW backward (the backward's recompute is not counted)
+        return 2.0 * s["M"] * s["d"] * s["V"] * (3.0 if bwd else 1.0)
     if kind == "grg":
         fwd = 2.0 * s["M"] * s["K"] * s["d"] + 2.0 * s["M"] * s["d"] * 2 * s["F"]
     else:
@@ -73,6 +76,8 @@ def _flops(kind, s, bwd):
 def _describe(name, kind, s, bwd):
     if kind == "grg":
         what = f"GEMM-Residual-RMSNorm-GEMM-SwiGLU {name} {'fwd+bwd' if bwd else 'fwd'}"
+    elif kind == "xent":
+        what = "LM-head cross-entropy fwd+bwd (LLaMA-3 vocabulary)"
     else:
         what = "SwiGLU MLP fwd+bwd"
     return {"workload": what, **s, "global_batch": s["M"]}
@@ -95,6 +100,12 @@ def _oracle_step(kind, s, bwd, inputs, rows):
     """The fp64 oracle over the first `rows` tokens of the workload (forward row-local,
     weight gradients summed over those rows only)."""
     from oracle import coda_oracle as O
+    if kind == "xent":
+        X, t, dl = inputs["X"][:rows], inputs["targets"][:rows], inputs["dloss"][:rows]
+        fwd = O.xent_forward(X, inputs["W"], t)
+        if bwd:
+            O.xent_backward(dl, X, inputs["W"], t, fwd=fwd)
+        return
     if kind == "grg":
         X, R, dY = inputs["X"][:rows], inputs["R"][:rows], inputs["dY"][:rows]
         fwd = O.grg_forward(X, inputs["W1"], R, inputs["g"], inputs["W2"], s["eps"])
@@ -113,6 +124,11 @@ def _oracle_inputs(kind, s):
     from gemm_epilogue_fusion_tmem_b200 import synth
     if kind == "grg":
         t = synth.grg_inputs(s["M"], s["K"], s["d"], s["F"], seed=0)
+    elif kind == "xent":
+        t = synth.xent_inputs(s["M"], s["d"], s["V"], seed=0)
+        out = {k: v.to(torch.float64).numpy() for k, v in t.items() if k != "targets"}
+        out["targets"] = t["targets"].long().numpy()
+        return out
     else:
         t = synth.swiglu_inputs(s["M"], s["d"], s["F"], seed=0)
     return {k: v.to(torch.float64).numpy() for k, v in t.items()}
@@ -253,6 +269,8 @@ def _setup(kind, s, bwd, device):
         host = synth.grg_inputs(s["M"], s["K"], s["d"], s["F"], seed=0)
         if not bwd:
             host.pop("dY")
+    elif kind == "xent":
+        host = synth.xent_inputs(s["M"], s["d"], s["V"], seed=0)
     else:
         host = synth.swiglu_inputs(s["M"], s["d"], s["F"], seed=0)
     dev = {k: v.to(device) for k, v in host.items()}
@@ -291,15 +309,27 @@ def _make_step(kind, s, bwd, dev):
         outs = {**fo, **bo}
         keys = ["Y", "dX", "dR", "dW1", "dW2", "dg"] if bwd else ["Y", "H", "r"]
         return step, outs, (10 if bwd else 4), keys, ws
+    if kind == "xent":
+        d, V = s["d"], s["V"]
+        ws = B.Workspace(max(lib.coda_xent_fwd_workspace_bytes(M, d, V), lib.coda_xent_bwd_workspace_bytes(M, d, V)),
+                         dev["X"].device)
+        fo = B.xent_fwd(dev["X"], dev["W"], dev["targets"], ws=ws)
+        bo = B.xent_bwd(dev["X"], dev["W"], dev["targets"], fo["lse"], dev["dloss"], ws=ws)
+
+        def xstep():
+            B.xent_fwd(dev["X"], dev["W"], dev["targets"], out=fo, ws=ws)
+            B.xent_bwd(dev["X"], dev["W"], dev["targets"], fo["lse"], dev["dloss"], out=bo, ws=ws)
+
+        return xstep, {**fo, **bo}, 5, ["loss", "dX", "dW"], ws
     d, F = s["d"], s["F"]
     ws = B.Workspace(lib.coda_swiglu_bwd_workspace_bytes(M, d, F), dev["X"].device)
-    fo, bo = {}, {}
+    fo = B.swiglu_fwd(dev["X"], dev["Wgu"], dev["Wdown"], ws=ws)
+    bo = B.swiglu_bwd(dev["dOut"], dev["X"], dev["Wgu"], dev["Wdown"], fo["Y"], fo["AB"], ws=ws)
 
     def step():
         B.swiglu_fwd(dev["X"], dev["Wgu"], dev["Wdown"], out=fo, ws=ws)
         B.swiglu_bwd(dev["dOut"], dev["X"], dev["Wgu"], dev["Wdown"], fo["Y"], fo["AB"], out=bo, ws=ws)
 
-    step()  # allocate outputs once
     outs = {**fo, **bo}
     return step, outs, 6, ["Out", "dX", "dWgu", "dWdown"], ws
 
@@ -329,9 +359,26 @@ def _make_unfused_step(s, bwd, dev):
 
 
 def _dominant_kernel(kind, s, dev, outs, reps=20):
-    """Time the dominant kernel alone: the gate/up GEMM with the r + SwiGLU epilogue."""
+    """Time the dominant kernel alone: the gate/up GEMM with the r + SwiGLU epilogue
+    (for the cross-entropy workload: the logits GEMM with its online-LSE epilogue)."""
     import torch
     from gemm_epilogue_fusion_tmem_b200 import binding as B
+    if kind == "xent":
+        lib = B.library()
+        M, d, V = s["M"], s["d"], s["V"]
+        ws = B.Workspace(lib.coda_xent_fwd_workspace_bytes(M, d, V), dev["X"].device)
+        o = {}
+        for _ in range(3):
+            B.xent_fwd(dev["X"], dev["W"], dev["targets"], out=o, ws=ws)
+        st = torch.cuda.current_stream()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(st)
+        for _ in range(reps):
+            B.xent_fwd(dev["X"], dev["W"], dev["targets"], out=o, ws=ws)
+        e1.record(st)
+        torch.cuda.synchronize()
+        return "xent_fwd (logits GEMM + online-LSE epilogue, row reduce)", e0.elapsed_time(e1) / reps, 2.0 * M * d * V
     if kind == "grg":
         A, W, r = outs["H"], dev["W2"], outs["r"]  # same shape and work as GEMM2 on W2g
         K = s["d"]

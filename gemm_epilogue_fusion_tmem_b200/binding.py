@@ -69,6 +69,10 @@ def library() -> ctypes.CDLL:
             "coda_swiglu_bwd": (I, [P, P, P, P, P, P, P, P, P, I, I, I, P, S, P]),
             "coda_grg_fwd_hg_workspace_bytes": (S, [I, I, I, I, I]),
             "coda_grg_fwd_hg": (I, [P] * 10 + [I, I, I, I, F, P, S, P]),
+            "coda_xent_fwd_workspace_bytes": (S, [I, I, I]),
+            "coda_xent_fwd": (I, [P, P, P, P, P, I, I, I, P, S, P]),
+            "coda_xent_bwd_workspace_bytes": (S, [I, I, I]),
+            "coda_xent_bwd": (I, [P, P, P, P, P, P, P, I, I, I, P, S, P]),
             "coda_grg_fwd_unfused_workspace_bytes": (S, [I, I, I, I]),
             "coda_grg_fwd_unfused": (I, [P] * 10 + [I, I, I, I, F, P, S, P]),
             "coda_grg_bwd_unfused_workspace_bytes": (S, [I, I, I, I]),
@@ -388,4 +392,41 @@ def grg_bwd_unfused(dY, X, W1, H, r, AB, U, g, W2, dH_in=None, out: dict | None 
                                     _ptr(g), _ptr(W2), _ptr(o["dX"]), _ptr(o["dR"]), _ptr(o["dW1"]), _ptr(o["dW2"]),
                                     _ptr(o["dg"]), M, K, d, N, ws.ptr(), ws.nbytes, _stream()),
            "coda_grg_bwd_unfused")
+    return o
+
+
+# ------------------------------------------------------------------ cross-entropy on the LM head
+
+def xent_fwd(X, W, targets, out: dict | None = None, ws: Workspace | None = None) -> dict:
+    """Per-row cross-entropy of X W^T without materialising the logits; returns loss, lse (fp32 [M])."""
+    lib = library()
+    M, d = X.shape
+    V = W.shape[0]
+    _req(X, "X"), _req(W, "W", shape=(V, d)), _req(targets, "targets", torch.int32, (M,))
+    o = dict(out or {})
+    for k in ("loss", "lse"):
+        if k not in o:
+            o[k] = torch.empty(M, dtype=torch.float32, device=X.device)
+        _req(o[k], k, torch.float32, (M,))
+    ws = ws or workspace(lib.coda_xent_fwd_workspace_bytes(M, d, V), X.device)
+    _check(lib.coda_xent_fwd(_ptr(X), _ptr(W), _ptr(targets), _ptr(o["loss"]), _ptr(o["lse"]), M, d, V,
+                             ws.ptr(), ws.nbytes, _stream()), "coda_xent_fwd")
+    return o
+
+
+def xent_bwd(X, W, targets, lse, dloss, out: dict | None = None, ws: Workspace | None = None) -> dict:
+    """Gradients of sum_i dloss_i loss_i; returns dX [M,d], dW [V,d] (bf16)."""
+    lib = library()
+    M, d = X.shape
+    V = W.shape[0]
+    _req(X, "X"), _req(W, "W", shape=(V, d)), _req(targets, "targets", torch.int32, (M,))
+    _req(lse, "lse", torch.float32, (M,)), _req(dloss, "dloss", torch.float32, (M,))
+    o = dict(out or {})
+    if "dX" not in o:
+        o["dX"] = torch.empty(M, d, dtype=torch.bfloat16, device=X.device)
+    if "dW" not in o:
+        o["dW"] = torch.empty(V, d, dtype=torch.bfloat16, device=X.device)
+    ws = ws or workspace(lib.coda_xent_bwd_workspace_bytes(M, d, V), X.device)
+    _check(lib.coda_xent_bwd(_ptr(X), _ptr(W), _ptr(targets), _ptr(lse), _ptr(dloss), _ptr(o["dX"]), _ptr(o["dW"]),
+                             M, d, V, ws.ptr(), ws.nbytes, _stream()), "coda_xent_bwd")
     return o

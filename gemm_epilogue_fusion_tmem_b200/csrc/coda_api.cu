@@ -26,7 +26,7 @@ inline int cdiv(long long a, long long b) { return (int)((a + b - 1) / b); }
 
 // ------------------------------------------------------------------ device checks
 
-constexpr int kKernelSlots = 48;  // (EPI, A major, B major, pair) instantiations
+constexpr int kKernelSlots = 64;  // (EPI, A major, B major, pair) instantiations: (7 * 4) * 2
 struct DevInfo {
   int num_sms = 0;
   int major = 0;
@@ -183,6 +183,7 @@ coda_status launch_gemm_mode(const CUtensorMap& ta, const CUtensorMap& tb, GemmP
   if (st != CODA_OK) return st;
   auto kern = gemm_tc_kernel<EPI, A_MN, B_MN, PAIR>;
   const int slot = ((EPI * 4 + (A_MN ? 2 : 0) + (B_MN ? 1 : 0)) * 2) + (PAIR ? 1 : 0);
+  static_assert(((EPI * 4 + 3) * 2 + 1) < kKernelSlots, "kernel slot table too small");
   DevInfo& di = g_dev[dev];
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof(cfg));
@@ -653,6 +654,98 @@ coda_status coda_swiglu_bwd(const void* dOut, const void* X, const void* Wgu, co
   CODA_TRY(gemm_store(dA, X, dWgu, 2 * F, d, M, true, true, nullptr, ws, s));
   CODA_TRY(gemm_store(dA, Wgu, dX, M, d, 2 * F, false, true, nullptr, ws, s));
   return CODA_OK;
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------ cross-entropy on the LM head
+
+extern "C" {
+
+size_t coda_xent_fwd_workspace_bytes(int M, int d, int V) {
+  (void)d;
+  if (M < 1 || V < 1) return kStatusBytes;
+  return kStatusBytes + align_up((size_t)M * cdiv(V, BN) * 8, 256) + align_up((size_t)M * 4, 256);
+}
+
+namespace {
+coda_status check_xent(const void* X, const void* W, const void* t, int M, int d, int V) {
+  if (!X || !W || !t) return CODA_ERR_INVALID_ARG;
+  if (M < 1 || d < 1 || V < 1) return CODA_ERR_INVALID_ARG;
+  if (d % 64 != 0 || V % 64 != 0) return CODA_ERR_UNSUPPORTED_SHAPE;
+  return CODA_OK;
+}
+}  // namespace
+
+coda_status coda_xent_fwd(const void* X, const void* W, const int32_t* targets, float* loss, float* lse, int M,
+                          int d, int V, void* ws, size_t ws_bytes, void* stream) {
+  CODA_TRY(check_xent(X, W, targets, M, d, V));
+  if (!loss || !lse || !ws) return CODA_ERR_INVALID_ARG;
+  const void* ptrs[] = {X, W, targets, loss, lse, ws};
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return CODA_ERR_MISALIGNED;
+  if (ws_bytes < coda_xent_fwd_workspace_bytes(M, d, V)) return CODA_ERR_WORKSPACE_TOO_SMALL;
+  int dev;
+  CODA_TRY(current_device(dev));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int T = cdiv(V, BN);
+  uint8_t* wsb = static_cast<uint8_t*>(ws) + kStatusBytes;
+  float* part = reinterpret_cast<float*>(wsb);
+  float* tlogit = reinterpret_cast<float*>(wsb + align_up((size_t)M * T * 8, 256));
+  // A target that no tile owns leaves NaN here, so its loss is NaN.
+  CODA_TRY(launch_status(cudaMemsetAsync(tlogit, 0xFF, (size_t)M * 4, s)));
+  {
+    const bool pair = use_pair();
+    CUtensorMap ta, tb;
+    if (!make_operand_map(&ta, X, M, d, false, BM) || !make_operand_map(&tb, W, V, d, false, pair ? BN / 2 : BN))
+      return CODA_ERR_CUDA;
+    GemmParams p = base_params(M, V, d, BN, ws, pair);
+    p.group_m = pick_group(M, V, d, p.num_m_tiles, p.num_n_tiles, pair, num_sms());
+    p.tgt = targets;
+    p.part = part;
+    p.ld_part = T;
+    p.outf = tlogit;
+    CODA_TRY((launch_gemm<EPI_XENT, false, false>(ta, tb, p, s, pair)));
+  }
+  return launch_status(launch_ex(xent_reduce_kernel, dim3(cdiv(M, 8)), dim3(256), 0, s, 1,
+                                 (const float2*)part, T, (const float*)tlogit, lse, loss, M));
+}
+
+size_t coda_xent_bwd_workspace_bytes(int M, int d, int V) {
+  (void)d;
+  if (M < 1 || V < 1) return kStatusBytes;
+  return kStatusBytes + align_up((size_t)M * V * 2, 256);
+}
+
+coda_status coda_xent_bwd(const void* X, const void* W, const int32_t* targets, const float* lse,
+                          const float* dloss, void* dX, void* dW, int M, int d, int V, void* ws, size_t ws_bytes,
+                          void* stream) {
+  CODA_TRY(check_xent(X, W, targets, M, d, V));
+  if (!lse || !dloss || !dX || !dW || !ws) return CODA_ERR_INVALID_ARG;
+  const void* ptrs[] = {X, W, targets, lse, dloss, dX, dW, ws};
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return CODA_ERR_MISALIGNED;
+  if (ws_bytes < coda_xent_bwd_workspace_bytes(M, d, V)) return CODA_ERR_WORKSPACE_TOO_SMALL;
+  int dev;
+  CODA_TRY(current_device(dev));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  __nv_bfloat16* dlogits = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(ws) + kStatusBytes);
+  {
+    const bool pair = use_pair();
+    CUtensorMap ta, tb;
+    if (!make_operand_map(&ta, X, M, d, false, BM) || !make_operand_map(&tb, W, V, d, false, pair ? BN / 2 : BN))
+      return CODA_ERR_CUDA;
+    GemmParams p = base_params(M, V, d, BN, ws, pair);
+    p.group_m = pick_group(M, V, d, p.num_m_tiles, p.num_n_tiles, pair, num_sms());
+    p.tgt = targets;
+    p.rowvec = lse;
+    p.rowvec2 = dloss;
+    p.out = dlogits;
+    p.ldo = V;
+    CODA_TRY((launch_gemm<EPI_XENT_BWD, false, false>(ta, tb, p, s, pair)));
+  }
+  CODA_TRY(gemm_store(dlogits, W, dX, M, d, V, false, true, nullptr, ws, s));
+  return gemm_store(dlogits, X, dW, V, d, M, true, true, nullptr, ws, s);
 }
 
 }  // extern "C"

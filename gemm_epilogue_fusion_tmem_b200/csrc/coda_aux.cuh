@@ -130,4 +130,43 @@ __global__ void __launch_bounds__(COLRED_THREADS)
   }
 }
 
+// Cross-entropy row reduce, one warp per row: merge the tiles' (max, sum exp)
+// partials, lse = max + log(sum), loss = lse - target logit (the target logit
+// is NaN when the target was out of range, so the loss is too).
+__device__ __forceinline__ void lse_merge(float& m, float& s, float om, float os) {
+  if (om == -INFINITY) return;
+  if (m == -INFINITY) {
+    m = om;
+    s = os;
+    return;
+  }
+  const float nm = fmaxf(m, om);
+  s = s * expf(m - nm) + os * expf(om - nm);
+  m = nm;
+}
+
+__global__ void xent_reduce_kernel(const float2* __restrict__ part, int T, const float* __restrict__ tlogit,
+                                   float* __restrict__ lse, float* __restrict__ loss, int M) {
+  griddep_wait();
+  const int row = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  const int lane = threadIdx.x & 31;
+  if (row >= M) return;
+  float m = -INFINITY, s = 0.f;
+  for (int t = lane; t < T; t += 32) {
+    const float2 q = part[(size_t)row * T + t];
+    lse_merge(m, s, q.x, q.y);
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    const float om = __shfl_xor_sync(0xffffffffu, m, o);
+    const float os = __shfl_xor_sync(0xffffffffu, s, o);
+    lse_merge(m, s, om, os);
+  }
+  if (lane == 0) {
+    const float l = m + logf(s);
+    lse[row] = l;
+    loss[row] = l - tlogit[row];
+  }
+}
+
 }  // namespace coda

@@ -38,6 +38,8 @@ enum Epi : int {
   EPI_SWIGLU = 2,      // a = r*acc_gate, b = r*acc_up; Y = silu(a)*b; AB = [a|b]
   EPI_DN = 3,          // dH = g*acc - c*H (+dH_in); column partials of acc*H
   EPI_SWIGLU_BWD = 4,  // dY = acc; da, db from a, b; dA = [da|db]
+  EPI_XENT = 5,        // logits tile: per-row online (max, sum exp) partials + the target logit
+  EPI_XENT_BWD = 6,    // dlogits = dloss_i (exp(logit - lse_i) - [j == t_i]), stored bf16
 };
 
 struct GemmParams {
@@ -61,6 +63,9 @@ struct GemmParams {
   int ld_part;
   __nv_bfloat16* out2;          // AB (SWIGLU), Hg (RESID_RMS), optional
   int ldo2;
+  const int* tgt;               // target class per row (XENT, XENT_BWD)
+  const float* rowvec2;         // dloss (XENT_BWD)
+  float* outf;                  // target logit per row (XENT)
   uint32_t* status;
   unsigned long long wait_limit_ns;
   uint32_t kernel_id;
@@ -237,6 +242,53 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbas
       for (int i = 0; i < 32; ++i) v[i] *= h[i];
       warp_column_sums(v, lane);
       p.part[(size_t)group32 * p.ld_part + n0 + c + lane] = v[0];
+    }
+  } else if constexpr (EPI == EPI_XENT) {
+    // Stateful transform (online max / sum-exp) over this tile's columns.
+    const int n0 = n_blk * BN;
+    const int t = rv ? p.tgt[row] : -1;
+    float m = -INFINITY, sum = 0.f, tl = 0.f;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      if (n0 + c >= p.N) break;
+      float v[32];
+      tmem_ld32(tbase + c, v);
+      float cm = v[0];
+#pragma unroll
+      for (int i = 1; i < 32; ++i) cm = fmaxf(cm, v[i]);
+      const float nm = fmaxf(m, cm);
+      float acc = 0.f;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) acc += __expf(v[i] - nm);
+      sum = sum * __expf(m - nm) + acc;
+      m = nm;
+      const int off = t - (n0 + c);
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (i == off) tl = v[i];
+    }
+    if (rv) {
+      reinterpret_cast<float2*>(p.part)[(size_t)row * p.ld_part + n_blk] = make_float2(m, sum);
+      if (t >= n0 && t < n0 + BN && t < p.N) p.outf[row] = tl;
+    }
+  } else if constexpr (EPI == EPI_XENT_BWD) {
+    const int n0 = n_blk * BN;
+    const int t = rv ? p.tgt[row] : -1;
+    const float lse = rv ? p.rowvec[row] : 0.f;
+    const float dl = rv ? p.rowvec2[row] : 0.f;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      if (n0 + c >= p.N) break;
+      float v[32];
+      tmem_ld32(tbase + c, v);
+      const int off = t - (n0 + c);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        float g = __expf(v[i] - lse);
+        if (i == off) g -= 1.f;
+        v[i] = g * dl;
+      }
+      if (rv) store32_bf16(p.out + (size_t)row * p.ldo + n0 + c, v);
     }
   } else if constexpr (EPI == EPI_SWIGLU_BWD) {
     const int n0 = n_blk * BN;

@@ -102,3 +102,17 @@ def gemm_inputs(M: int, N: int, K: int, seed: int = 0) -> dict:
     """A[M,K], B[N,K] ~ N(0,1) bf16 for plain-GEMM checks."""
     gen = torch.Generator().manual_seed(seed)
     return {"A": _normal(gen, (M, K)), "B": _normal(gen, (N, K), std=K ** -0.5)}
+
+
+def xent_inputs(M: int, d: int, V: int, seed: int = 0) -> dict:
+    """LM-head inputs drawn in the order X, W, targets, dloss: X ~ N(0,1), W ~ N(0, 1/d),
+    targets uniform in [0, V) (int32), dloss ~ U(0, 1) / M (fp32)."""
+    gen = torch.Generator().manual_seed(seed)
+    X = _normal(gen, (M, d))
+    W = _normal(gen, (V, d), std=d ** -0.5)
+    targets = torch.randint(0, V, (M,), generator=gen, dtype=torch.int64).to(torch.int32)
+    dloss = torch.rand(M, generator=gen, dtype=torch.float32) / M
+    return {"X": X, "W": W, "targets": targets, "dloss": dloss}
+
+
+XENT_LM_HEAD = {"name": "xent", "M": 8192, "d": 4096, "V": 128256}

@@ -216,6 +216,36 @@ coda_status coda_swiglu_bwd(const void* dOut, const void* X, const void* Wgu, co
                             void* dX, void* dWgu, void* dWdown,
                             int M, int d, int F, void* ws, size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------- cross-entropy on the LM head */
+
+/* Workspace for coda_xent_fwd: status word, per-tile (max, sum exp) partials
+ * [M, ceil(V/256)] float2 and the target logits [M] fp32. */
+size_t coda_xent_fwd_workspace_bytes(int M, int d, int V);
+
+/* Cross-entropy of logits = X W^T without writing the logits to HBM: the
+ * LM-head GEMM's epilogue keeps, per row and 256-column tile, the online
+ * maximum and sum of exponentials (the stateful transform and tile-wise
+ * log-sum-exp of the toolin.ai five-primitive table) and picks out the target
+ * logit; a warp-per-row reduce merges the tiles:
+ *   lse_i = log sum_j exp(logits_ij),  loss_i = lse_i - logits_i,t_i.
+ * Inputs X [M,d] bf16, W [V,d] bf16, targets [M] int32 in [0, V).
+ * Outputs loss [M] and lse [M] fp32 (loss is NaN for an out-of-range target).
+ * Requires M >= 1, d % 64 == 0, V % 64 == 0.  Logits are fp32 accumulators. */
+coda_status coda_xent_fwd(const void* X, const void* W, const int32_t* targets, float* loss, float* lse,
+                          int M, int d, int V, void* ws, size_t ws_bytes, void* stream);
+
+/* Workspace for coda_xent_bwd: status word and dlogits [M, V] bf16. */
+size_t coda_xent_bwd_workspace_bytes(int M, int d, int V);
+
+/* Backward of sum_i dloss_i loss_i.  The GEMM is recomputed and its epilogue
+ * writes dlogits_ij = dloss_i (exp(logits_ij - lse_i) - [j == t_i]) (bf16);
+ * then dX = dlogits W and dW = dlogits^T X (plain GEMMs).
+ * Inputs X, W, targets as coda_xent_fwd, lse [M] from it, dloss [M] fp32.
+ * Outputs dX [M,d], dW [V,d] bf16.  Same shape rules. */
+coda_status coda_xent_bwd(const void* X, const void* W, const int32_t* targets, const float* lse,
+                          const float* dloss, void* dX, void* dW, int M, int d, int V,
+                          void* ws, size_t ws_bytes, void* stream);
+
 /* ---------------------------------------------------------------- unfused comparison sequence */
 
 /* The same block run operator by operator, the way a framework without
