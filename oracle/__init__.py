@@ -10,6 +10,10 @@ from .coda_oracle import (  # noqa: F401
     grg_backward,
     grg_forward,
     partial_sumsq,
+    qkv_rope_backward,
+    qkv_rope_forward,
+    rope_angles,
+    rope_rotate,
     silu,
     swiglu_backward,
     swiglu_forward,

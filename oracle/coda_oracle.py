@@ -57,6 +57,10 @@ __all__ = [
     "swiglu_backward_stored",
     "xent_forward",
     "xent_backward",
+    "rope_angles",
+    "rope_rotate",
+    "qkv_rope_forward",
+    "qkv_rope_backward",
 ]
 
 
@@ -364,3 +368,66 @@ def xent_backward(dloss, X, W, targets, fwd: dict | None = None, store=None) -> 
     if store is not None:
         dlogits = store(dlogits)
     return {"dlogits": dlogits, "dX": dlogits @ W, "dW": dlogits.T @ X}
+
+
+# ----------------------------------------------------------------------------- rotary position embedding
+
+def rope_angles(seq_len: int, head_dim: int, base: float) -> np.ndarray:
+    """angle[pos, j] = pos * base^(-2j / head_dim), j in [0, head_dim / 2)."""
+    j = np.arange(head_dim // 2, dtype=np.float64)
+    inv_freq = base ** (-2.0 * j / head_dim)
+    return np.arange(seq_len, dtype=np.float64)[:, None] * inv_freq[None, :]
+
+
+def rope_rotate(x, positions, head_dim: int, base: float, inverse: bool = False) -> np.ndarray:
+    """Rotate each head of x [M, heads*head_dim]: the pair (j, j + head_dim/2)
+    of a head at position p turns by p * base^(-2j/head_dim) (the
+    rotate-half pairing); inverse=True turns by the negative angle."""
+    x = _f64(x)
+    M, W = x.shape
+    half = head_dim // 2
+    ang = np.asarray(positions, dtype=np.float64)[:, None] * \
+        (base ** (-2.0 * np.arange(half, dtype=np.float64) / head_dim))[None, :]
+    if inverse:
+        ang = -ang
+    c, s = np.cos(ang), np.sin(ang)
+    out = np.empty_like(x)
+    for h in range(W // head_dim):
+        x1 = x[:, h * head_dim:h * head_dim + half]
+        x2 = x[:, h * head_dim + half:(h + 1) * head_dim]
+        out[:, h * head_dim:h * head_dim + half] = x1 * c - x2 * s
+        out[:, h * head_dim + half:(h + 1) * head_dim] = x2 * c + x1 * s
+    return out
+
+
+def qkv_rope_forward(X, Wqkv, n_q: int, n_kv: int, head_dim: int, seq_len: int, base: float) -> dict:
+    """QKV projection followed by RoPE on the q and k heads, unfused.
+
+      QKV = X Wqkv^T, columns [q heads | k heads | v heads] (n_q, n_kv, n_kv heads)
+      q, k rotated at position pos = token index mod seq_len; v unchanged.
+    RoPE is one of the elementwise transforms the pages place in a GEMM
+    epilogue (toolin.ai five-primitive table, row "elementwise transform";
+    kucoin (ru) «В «Финале» спрятаны сокровища»).
+    """
+    X, Wqkv = _f64(X), _f64(Wqkv)
+    pre = X @ Wqkv.T
+    pos = np.arange(X.shape[0]) % seq_len
+    nqk = (n_q + n_kv) * head_dim
+    out = pre.copy()
+    out[:, :nqk] = rope_rotate(pre[:, :nqk], pos, head_dim, base)
+    return {"pre": pre, "QKV": out}
+
+
+def qkv_rope_backward(dQKV, X, Wqkv, n_q: int, n_kv: int, head_dim: int, seq_len: int, base: float,
+                      store=None) -> dict:
+    """Gradients of <dQKV, QKV>: the inverse rotation of the q/k gradient, then
+    dX = dPre Wqkv and dW = dPre^T X (store: optional rounding of dPre, which
+    the method stores as bf16 before the GEMMs read it)."""
+    dQKV, X, Wqkv = _f64(dQKV), _f64(X), _f64(Wqkv)
+    pos = np.arange(X.shape[0]) % seq_len
+    nqk = (n_q + n_kv) * head_dim
+    dpre = dQKV.copy()
+    dpre[:, :nqk] = rope_rotate(dQKV[:, :nqk], pos, head_dim, base, inverse=True)
+    if store is not None:
+        dpre = store(dpre)
+    return {"dpre": dpre, "dX": dpre @ Wqkv, "dW": dpre.T @ X}

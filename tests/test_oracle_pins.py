@@ -411,3 +411,57 @@ def test_xent_shift_invariance_and_finite_differences():
     p = {"X": X.copy(), "W": W.copy()}
     _fd_check(lambda q: float(np.sum(dloss * O.xent_forward(q["X"], q["W"], t)["loss"])), p,
               {"X": b["dX"], "W": b["dW"]}, ["X", "W"])
+
+
+# ----------------------------------------------------------------------------- RoPE
+
+def test_rope_closed_forms():
+    """head_dim 2: the single pair turns by exactly pos radians (base^0 = 1); pos 0 is the identity."""
+    x = np.array([[1.0, 0.0], [1.0, 0.0], [0.0, 2.0], [3.0, -1.0]])
+    pos = np.array([0, 1, 2, 0])
+    y = O.rope_rotate(x, pos, head_dim=2, base=10000.0)
+    np.testing.assert_allclose(y[0], [1.0, 0.0], atol=1e-15)
+    np.testing.assert_allclose(y[1], [np.cos(1.0), np.sin(1.0)], rtol=1e-15)
+    np.testing.assert_allclose(y[2], [-2.0 * np.sin(2.0), 2.0 * np.cos(2.0)], rtol=1e-14)
+    np.testing.assert_allclose(y[3], [3.0, -1.0], atol=1e-15)
+    # Second frequency of head_dim 4 with base 100: 100^(-2/4) = 0.1 rad per position.
+    z = O.rope_rotate(np.array([[0.0, 1.0, 0.0, 0.0]]), np.array([5]), head_dim=4, base=100.0)
+    np.testing.assert_allclose(z[0], [0.0, np.cos(0.5), 0.0, np.sin(0.5)], atol=1e-15)
+
+
+def test_rope_preserves_norms_and_inverse_undoes_it():
+    rng = np.random.default_rng(19)
+    M, heads, hd = 9, 3, 8
+    x = rng.standard_normal((M, heads * hd))
+    pos = rng.integers(0, 4096, M)
+    y = O.rope_rotate(x, pos, hd, 10000.0)
+    for h in range(heads):
+        np.testing.assert_allclose(np.linalg.norm(y[:, h * hd:(h + 1) * hd], axis=1),
+                                   np.linalg.norm(x[:, h * hd:(h + 1) * hd], axis=1), rtol=1e-13)
+    np.testing.assert_allclose(O.rope_rotate(y, pos, hd, 10000.0, inverse=True), x, atol=1e-12)
+
+
+def test_rope_relative_position_property():
+    """<RoPE(q, m), RoPE(k, n)> depends on m - n only: RoPE's defining property."""
+    rng = np.random.default_rng(20)
+    hd = 16
+    q, k = rng.standard_normal((1, hd)), rng.standard_normal((1, hd))
+    dots = []
+    for m, n in [(7, 3), (104, 100), (4004, 4000)]:
+        qm = O.rope_rotate(q, np.array([m]), hd, 10000.0)
+        kn = O.rope_rotate(k, np.array([n]), hd, 10000.0)
+        dots.append(float((qm @ kn.T)[0, 0]))
+    np.testing.assert_allclose(dots, dots[0], rtol=1e-10)
+
+
+def test_qkv_rope_backward_finite_differences():
+    rng = np.random.default_rng(21)
+    M, d, nq, nkv, hd, S = 5, 6, 2, 1, 4, 3
+    p = {"X": rng.standard_normal((M, d)), "W": rng.standard_normal(((nq + 2 * nkv) * hd, d))}
+    dQ = rng.standard_normal((M, (nq + 2 * nkv) * hd))
+    b = O.qkv_rope_backward(dQ, p["X"], p["W"], nq, nkv, hd, S, 50.0)
+    _fd_check(lambda q: float(np.sum(dQ * O.qkv_rope_forward(q["X"], q["W"], nq, nkv, hd, S, 50.0)["QKV"])),
+              p, {"X": b["dX"], "W": b["dW"]}, ["X", "W"])
+    # v columns pass through unrotated.
+    f = O.qkv_rope_forward(p["X"], p["W"], nq, nkv, hd, S, 50.0)
+    np.testing.assert_array_equal(f["QKV"][:, (nq + nkv) * hd:], f["pre"][:, (nq + nkv) * hd:])
