@@ -39,6 +39,7 @@ WORKLOADS = {
     "70B": ("grg", dict(M=4096, K=8192, d=8192, F=28672, eps=1e-5), True),
     "swiglu": ("swiglu", dict(M=16384, d=4096, F=14336), True),
     "xent": ("xent", dict(M=8192, d=4096, V=128256), True),
+    "rope": ("rope", dict(M=8192, d=4096, n_q=32, n_kv=32, head_dim=128, seq_len=2048, base=10000.0), True),
 }
 
 
@@ -64,6 +65,8 @@ def _peaks():
 
 
 def _flops(kind, s, bwd):
+    if kind == "rope":
+        return 2.0 * s["M"] * s["d"] * (s["n_q"] + 2 * s["n_kv"]) * s["head_dim"] * (3.0 if bwd else 1.0)
     if kind == "xent":  # logits GEMM forward, dX and dW backward (the backward's recompute is not counted)
         return 2.0 * s["M"] * s["d"] * s["V"] * (3.0 if bwd else 1.0)
     if kind == "grg":
@@ -78,6 +81,8 @@ def _describe(name, kind, s, bwd):
         what = f"GEMM-Residual-RMSNorm-GEMM-SwiGLU {name} {'fwd+bwd' if bwd else 'fwd'}"
     elif kind == "xent":
         what = "LM-head cross-entropy fwd+bwd (LLaMA-3 vocabulary)"
+    elif kind == "rope":
+        what = "QKV projection with RoPE epilogue fwd+bwd (LLaMA-7B attention)"
     else:
         what = "SwiGLU MLP fwd+bwd"
     return {"workload": what, **s, "global_batch": s["M"]}
@@ -100,6 +105,13 @@ def _oracle_step(kind, s, bwd, inputs, rows):
     """The fp64 oracle over the first `rows` tokens of the workload (forward row-local,
     weight gradients summed over those rows only)."""
     from oracle import coda_oracle as O
+    if kind == "rope":
+        X = inputs["X"][:rows]
+        a = (s["n_q"], s["n_kv"], s["head_dim"], s["seq_len"], s["base"])
+        O.qkv_rope_forward(X, inputs["Wqkv"], *a)
+        if bwd:
+            O.qkv_rope_backward(inputs["dQKV"][:rows], X, inputs["Wqkv"], *a)
+        return
     if kind == "xent":
         X, t, dl = inputs["X"][:rows], inputs["targets"][:rows], inputs["dloss"][:rows]
         fwd = O.xent_forward(X, inputs["W"], t)
@@ -124,6 +136,8 @@ def _oracle_inputs(kind, s):
     from gemm_epilogue_fusion_tmem_b200 import synth
     if kind == "grg":
         t = synth.grg_inputs(s["M"], s["K"], s["d"], s["F"], seed=0)
+    elif kind == "rope":
+        t = synth.qkv_inputs(s["M"], s["d"], s["n_q"], s["n_kv"], s["head_dim"], seed=0)
     elif kind == "xent":
         t = synth.xent_inputs(s["M"], s["d"], s["V"], seed=0)
         out = {k: v.to(torch.float64).numpy() for k, v in t.items() if k != "targets"}
@@ -271,6 +285,8 @@ def _setup(kind, s, bwd, device):
             host.pop("dY")
     elif kind == "xent":
         host = synth.xent_inputs(s["M"], s["d"], s["V"], seed=0)
+    elif kind == "rope":
+        host = synth.qkv_inputs(s["M"], s["d"], s["n_q"], s["n_kv"], s["head_dim"], seed=0)
     else:
         host = synth.swiglu_inputs(s["M"], s["d"], s["F"], seed=0)
     dev = {k: v.to(device) for k, v in host.items()}
@@ -309,6 +325,18 @@ def _make_step(kind, s, bwd, dev):
         outs = {**fo, **bo}
         keys = ["Y", "dX", "dR", "dW1", "dW2", "dg"] if bwd else ["Y", "H", "r"]
         return step, outs, (10 if bwd else 4), keys, ws
+    if kind == "rope":
+        a = (s["n_q"], s["n_kv"], s["head_dim"], s["seq_len"], s["base"])
+        ws = B.Workspace(lib.coda_qkv_rope_bwd_workspace_bytes(M, s["d"], s["n_q"], s["n_kv"], s["head_dim"]),
+                         dev["X"].device)
+        q = B.qkv_rope_fwd(dev["X"], dev["Wqkv"], *a, ws=ws)
+        bo = B.qkv_rope_bwd(dev["dQKV"], dev["X"], dev["Wqkv"], *a, ws=ws)
+
+        def rstep():
+            B.qkv_rope_fwd(dev["X"], dev["Wqkv"], *a, out=q, ws=ws)
+            B.qkv_rope_bwd(dev["dQKV"], dev["X"], dev["Wqkv"], *a, out=bo, ws=ws)
+
+        return rstep, {"QKV": q, **bo}, 4, ["QKV", "dX", "dW"], ws
     if kind == "xent":
         d, V = s["d"], s["V"]
         ws = B.Workspace(max(lib.coda_xent_fwd_workspace_bytes(M, d, V), lib.coda_xent_bwd_workspace_bytes(M, d, V)),
@@ -363,6 +391,21 @@ def _dominant_kernel(kind, s, dev, outs, reps=20):
     (for the cross-entropy workload: the logits GEMM with its online-LSE epilogue)."""
     import torch
     from gemm_epilogue_fusion_tmem_b200 import binding as B
+    if kind == "rope":
+        a = (s["n_q"], s["n_kv"], s["head_dim"], s["seq_len"], s["base"])
+        q = outs["QKV"]
+        for _ in range(3):
+            B.qkv_rope_fwd(dev["X"], dev["Wqkv"], *a, out=q)
+        st = torch.cuda.current_stream()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(st)
+        for _ in range(reps):
+            B.qkv_rope_fwd(dev["X"], dev["Wqkv"], *a, out=q)
+        e1.record(st)
+        torch.cuda.synchronize()
+        return ("qkv_rope_fwd (QKV GEMM + RoPE epilogue)", e0.elapsed_time(e1) / reps,
+                2.0 * s["M"] * s["d"] * (s["n_q"] + 2 * s["n_kv"]) * s["head_dim"])
     if kind == "xent":
         lib = B.library()
         M, d, V = s["M"], s["d"], s["V"]

@@ -73,6 +73,9 @@ def library() -> ctypes.CDLL:
             "coda_xent_fwd": (I, [P, P, P, P, P, I, I, I, P, S, P]),
             "coda_xent_bwd_workspace_bytes": (S, [I, I, I]),
             "coda_xent_bwd": (I, [P, P, P, P, P, P, P, I, I, I, P, S, P]),
+            "coda_qkv_rope_fwd": (I, [P, P, P, I, I, I, I, I, I, F, P, S, P]),
+            "coda_qkv_rope_bwd_workspace_bytes": (S, [I, I, I, I, I]),
+            "coda_qkv_rope_bwd": (I, [P, P, P, P, P, I, I, I, I, I, I, F, P, S, P]),
             "coda_grg_fwd_unfused_workspace_bytes": (S, [I, I, I, I]),
             "coda_grg_fwd_unfused": (I, [P] * 10 + [I, I, I, I, F, P, S, P]),
             "coda_grg_bwd_unfused_workspace_bytes": (S, [I, I, I, I]),
@@ -429,4 +432,39 @@ def xent_bwd(X, W, targets, lse, dloss, out: dict | None = None, ws: Workspace |
     ws = ws or workspace(lib.coda_xent_bwd_workspace_bytes(M, d, V), X.device)
     _check(lib.coda_xent_bwd(_ptr(X), _ptr(W), _ptr(targets), _ptr(lse), _ptr(dloss), _ptr(o["dX"]), _ptr(o["dW"]),
                              M, d, V, ws.ptr(), ws.nbytes, _stream()), "coda_xent_bwd")
+    return o
+
+
+# ------------------------------------------------------------------ QKV projection with RoPE
+
+def qkv_rope_fwd(X, Wqkv, n_q: int, n_kv: int, head_dim: int, seq_len: int, base: float = 10000.0,
+                 out: torch.Tensor | None = None, ws: Workspace | None = None) -> torch.Tensor:
+    """QKV = X Wqkv^T with RoPE on the q and k heads applied in the GEMM epilogue."""
+    lib = library()
+    M, d = X.shape
+    ncols = (n_q + 2 * n_kv) * head_dim
+    _req(X, "X"), _req(Wqkv, "Wqkv", shape=(ncols, d))
+    Q = out if out is not None else torch.empty(M, ncols, dtype=torch.bfloat16, device=X.device)
+    _req(Q, "QKV", shape=(M, ncols))
+    ws = ws or workspace(lib.coda_gemm_workspace_bytes(), X.device)
+    _check(lib.coda_qkv_rope_fwd(_ptr(X), _ptr(Wqkv), _ptr(Q), M, d, n_q, n_kv, head_dim, seq_len, float(base),
+                                 ws.ptr(), ws.nbytes, _stream()), "coda_qkv_rope_fwd")
+    return Q
+
+
+def qkv_rope_bwd(dQKV, X, Wqkv, n_q: int, n_kv: int, head_dim: int, seq_len: int, base: float = 10000.0,
+                 out: dict | None = None, ws: Workspace | None = None) -> dict:
+    """Backward of qkv_rope_fwd; returns dX, dW."""
+    lib = library()
+    M, d = X.shape
+    ncols = (n_q + 2 * n_kv) * head_dim
+    _req(dQKV, "dQKV", shape=(M, ncols)), _req(X, "X"), _req(Wqkv, "Wqkv", shape=(ncols, d))
+    o = dict(out or {})
+    if "dX" not in o:
+        o["dX"] = torch.empty(M, d, dtype=torch.bfloat16, device=X.device)
+    if "dW" not in o:
+        o["dW"] = torch.empty(ncols, d, dtype=torch.bfloat16, device=X.device)
+    ws = ws or workspace(lib.coda_qkv_rope_bwd_workspace_bytes(M, d, n_q, n_kv, head_dim), X.device)
+    _check(lib.coda_qkv_rope_bwd(_ptr(dQKV), _ptr(X), _ptr(Wqkv), _ptr(o["dX"]), _ptr(o["dW"]), M, d, n_q, n_kv,
+                                 head_dim, seq_len, float(base), ws.ptr(), ws.nbytes, _stream()), "coda_qkv_rope_bwd")
     return o

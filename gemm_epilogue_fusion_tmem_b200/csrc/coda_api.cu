@@ -37,6 +37,8 @@ DevInfo g_dev[64];
 
 int g_last_sms = 148;
 int num_sms() { return g_last_sms; }
+// Grid for grid-stride elementwise kernels over n_vec8 8-element vectors.
+inline int ew_grid(long long n_vec8) { return (int)std::min<long long>(cdiv(n_vec8, 256), (long long)num_sms() * 16); }
 
 coda_status current_device(int& dev) {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return CODA_ERR_CUDA;
@@ -750,13 +752,82 @@ coda_status coda_xent_bwd(const void* X, const void* W, const int32_t* targets, 
 
 }  // extern "C"
 
-// ------------------------------------------------------------------ unfused comparison sequence
+// ------------------------------------------------------------------ QKV projection with RoPE
 
 namespace coda {
 namespace {
-inline int ew_grid(long long n_vec8) { return (int)std::min<long long>(cdiv(n_vec8, 256), (long long)num_sms() * 16); }
+coda_status check_rope(const void* X, const void* W, int M, int d, int n_q, int n_kv, int head_dim, int seq_len,
+                       float base) {
+  if (!X || !W) return CODA_ERR_INVALID_ARG;
+  if (M < 1 || d < 1 || n_q < 1 || n_kv < 1 || seq_len < 1 || !(base > 1.f)) return CODA_ERR_INVALID_ARG;
+  if (d % 64 != 0 || !(head_dim == 64 || head_dim == 128 || head_dim == 256)) return CODA_ERR_UNSUPPORTED_SHAPE;
+  return CODA_OK;
+}
+float rope_k(int head_dim, float base) { return -2.0f * log2f(base) / (float)head_dim; }
 }  // namespace
 }  // namespace coda
+
+extern "C" {
+
+coda_status coda_qkv_rope_fwd(const void* X, const void* Wqkv, void* QKV, int M, int d, int n_q, int n_kv,
+                              int head_dim, int seq_len, float base, void* ws, size_t ws_bytes, void* stream) {
+  CODA_TRY(check_rope(X, Wqkv, M, d, n_q, n_kv, head_dim, seq_len, base));
+  if (!QKV || !ws) return CODA_ERR_INVALID_ARG;
+  const void* ptrs[] = {X, Wqkv, QKV, ws};
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return CODA_ERR_MISALIGNED;
+  if (ws_bytes < coda_gemm_workspace_bytes()) return CODA_ERR_WORKSPACE_TOO_SMALL;
+  int dev;
+  CODA_TRY(current_device(dev));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int ncols = (n_q + 2 * n_kv) * head_dim;
+  const bool pair = use_pair();
+  CUtensorMap ta, tb;
+  if (!make_operand_map(&ta, X, M, d, false, BM) || !make_operand_map(&tb, Wqkv, ncols, d, false, pair ? BN / 2 : BN))
+    return CODA_ERR_CUDA;
+  GemmParams p = base_params(M, ncols, d, BN, ws, pair);
+  p.group_m = pick_group(M, ncols, d, p.num_m_tiles, p.num_n_tiles, pair, num_sms());
+  p.out = bf(QKV);
+  p.ldo = ncols;
+  p.head_dim = head_dim;
+  p.rot_cols = (n_q + n_kv) * head_dim;
+  p.seq_len = seq_len;
+  p.rope_k = rope_k(head_dim, base);
+  return launch_gemm<EPI_ROPE, false, false>(ta, tb, p, s, pair);
+}
+
+size_t coda_qkv_rope_bwd_workspace_bytes(int M, int d, int n_q, int n_kv, int head_dim) {
+  (void)d;
+  if (M < 1 || n_q < 1 || n_kv < 1 || head_dim < 1) return kStatusBytes;
+  return kStatusBytes + align_up((size_t)M * (n_q + 2 * n_kv) * head_dim * 2, 256);
+}
+
+coda_status coda_qkv_rope_bwd(const void* dQKV, const void* X, const void* Wqkv, void* dX, void* dW, int M, int d,
+                              int n_q, int n_kv, int head_dim, int seq_len, float base, void* ws, size_t ws_bytes,
+                              void* stream) {
+  CODA_TRY(check_rope(X, Wqkv, M, d, n_q, n_kv, head_dim, seq_len, base));
+  if (!dQKV || !dX || !dW || !ws) return CODA_ERR_INVALID_ARG;
+  const void* ptrs[] = {dQKV, X, Wqkv, dX, dW, ws};
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return CODA_ERR_MISALIGNED;
+  if (ws_bytes < coda_qkv_rope_bwd_workspace_bytes(M, d, n_q, n_kv, head_dim)) return CODA_ERR_WORKSPACE_TOO_SMALL;
+  int dev;
+  CODA_TRY(current_device(dev));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int ncols = (n_q + 2 * n_kv) * head_dim;
+  __nv_bfloat16* dpre = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(ws) + kStatusBytes);
+  const int rot_cols = (n_q + n_kv) * head_dim;
+  const long long items = (long long)M * ((rot_cols / head_dim) * (head_dim / 16) + (ncols - rot_cols) / 8);
+  CODA_TRY(launch_status(launch_ex(rope_unrotate_kernel, dim3(ew_grid(items)), dim3(256), 0, s, 1, cbf(dQKV),
+                                   dpre, M, ncols, head_dim, rot_cols, seq_len, rope_k(head_dim, base))));
+  CODA_TRY(gemm_store(dpre, Wqkv, dX, M, d, ncols, false, true, nullptr, ws, s));
+  return gemm_store(dpre, X, dW, ncols, d, M, true, true, nullptr, ws, s);
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------ unfused comparison sequence
+
 
 extern "C" {
 

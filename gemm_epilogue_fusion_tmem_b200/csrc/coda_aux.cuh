@@ -133,6 +133,47 @@ __global__ void __launch_bounds__(COLRED_THREADS)
 // Cross-entropy row reduce, one warp per row: merge the tiles' (max, sum exp)
 // partials, lse = max + log(sum), loss = lse - target logit (the target logit
 // is NaN when the target was out of range, so the loss is too).
+// Inverse RoPE of the q/k gradient (rotation by -pos * base^(-2j/hd)) and a
+// copy of the v gradient, 8 pairs (or 8 v columns) per thread:
+// dpre = R(pos)^T dQKV, the A operand of the backward GEMMs.
+__global__ void rope_unrotate_kernel(const __nv_bfloat16* __restrict__ dq, __nv_bfloat16* __restrict__ dpre,
+                                     int M, int ncols, int head_dim, int rot_cols, int seq_len, float rope_k) {
+  griddep_wait();
+  const int half = head_dim / 2;
+  const int rot_items = (rot_cols / head_dim) * (half / 8);
+  const int per_row = rot_items + (ncols - rot_cols) / 8;
+  const long long total = (long long)M * per_row;
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  for (long long it = (long long)blockIdx.x * blockDim.x + threadIdx.x; it < total; it += stride) {
+    const int row = (int)(it / per_row);
+    const int k = (int)(it - (long long)row * per_row);
+    const size_t base = (size_t)row * ncols;
+    if (k >= rot_items) {
+      const int c = rot_cols + (k - rot_items) * 8;
+      stg_v4(dpre + base + c, ldg_nc_v4(dq + base + c));
+      continue;
+    }
+    const int h = k / (half / 8);
+    const int j0 = (k - h * (half / 8)) * 8;
+    const int c1 = h * head_dim + j0;
+    float x1[8], x2[8];
+    unpack8(ldg_nc_v4(dq + base + c1), x1);
+    unpack8(ldg_nc_v4(dq + base + c1 + half), x2);
+    const float pos = (float)(row % seq_len);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float sn, cs;
+      sincosf(pos * exp2f((float)(j0 + i) * rope_k), &sn, &cs);
+      const float y1 = x1[i] * cs + x2[i] * sn;
+      const float y2 = x2[i] * cs - x1[i] * sn;
+      x1[i] = y1;
+      x2[i] = y2;
+    }
+    stg_v4(dpre + base + c1, pack8(x1));
+    stg_v4(dpre + base + c1 + half, pack8(x2));
+  }
+}
+
 __device__ __forceinline__ void lse_merge(float& m, float& s, float om, float os) {
   if (om == -INFINITY) return;
   if (m == -INFINITY) {

@@ -40,6 +40,7 @@ enum Epi : int {
   EPI_SWIGLU_BWD = 4,  // dY = acc; da, db from a, b; dA = [da|db]
   EPI_XENT = 5,        // logits tile: per-row online (max, sum exp) partials + the target logit
   EPI_XENT_BWD = 6,    // dlogits = dloss_i (exp(logit - lse_i) - [j == t_i]), stored bf16
+  EPI_ROPE = 7,        // QKV tile: rotate the q/k heads' (j, j + hd/2) pairs by pos * base^(-2j/hd)
 };
 
 struct GemmParams {
@@ -66,6 +67,10 @@ struct GemmParams {
   const int* tgt;               // target class per row (XENT, XENT_BWD)
   const float* rowvec2;         // dloss (XENT_BWD)
   float* outf;                  // target logit per row (XENT)
+  int head_dim;                 // ROPE: head width (64, 128 or 256)
+  int rot_cols;                 // ROPE: columns [0, rot_cols) are rotated (q and k heads)
+  int seq_len;                  // ROPE: position = row % seq_len
+  float rope_k;                 // ROPE: -2 log2(base) / head_dim, so inv_freq_j = 2^(j * rope_k)
   uint32_t* status;
   unsigned long long wait_limit_ns;
   uint32_t kernel_id;
@@ -289,6 +294,37 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbas
         v[i] = g * dl;
       }
       if (rv) store32_bf16(p.out + (size_t)row * p.ldo + n0 + c, v);
+    }
+  } else if constexpr (EPI == EPI_ROPE) {
+    const int n0 = n_blk * BN;
+    const float pos = (float)(row % p.seq_len);
+    const int half = p.head_dim / 2;
+#pragma unroll 1
+    for (int h0 = 0; h0 < BN; h0 += p.head_dim) {
+      const int col0 = n0 + h0;
+      if (col0 >= p.N) break;
+      const bool rot = col0 < p.rot_cols;
+#pragma unroll 1
+      for (int c = 0; c < half; c += 32) {
+        float x1[32], x2[32];
+        tmem_ld32(tbase + h0 + c, x1);
+        tmem_ld32(tbase + h0 + half + c, x2);
+        if (rot) {
+#pragma unroll 4
+          for (int i = 0; i < 32; ++i) {
+            float sn, cs;
+            sincosf(pos * exp2f((float)(c + i) * p.rope_k), &sn, &cs);
+            const float y1 = x1[i] * cs - x2[i] * sn;
+            const float y2 = x2[i] * cs + x1[i] * sn;
+            x1[i] = y1;
+            x2[i] = y2;
+          }
+        }
+        if (rv) {
+          store32_bf16(p.out + (size_t)row * p.ldo + col0 + c, x1);
+          store32_bf16(p.out + (size_t)row * p.ldo + col0 + half + c, x2);
+        }
+      }
     }
   } else if constexpr (EPI == EPI_SWIGLU_BWD) {
     const int n0 = n_blk * BN;

@@ -116,3 +116,17 @@ def xent_inputs(M: int, d: int, V: int, seed: int = 0) -> dict:
 
 
 XENT_LM_HEAD = {"name": "xent", "M": 8192, "d": 4096, "V": 128256}
+
+
+def qkv_inputs(M: int, d: int, n_q: int, n_kv: int, head_dim: int, seed: int = 0) -> dict:
+    """QKV projection inputs drawn in the order X, Wqkv, dQKV: X ~ N(0,1),
+    Wqkv ~ N(0, 1/d) with rows [q heads | k heads | v heads], dQKV ~ N(0,1)."""
+    gen = torch.Generator().manual_seed(seed)
+    ncols = (n_q + 2 * n_kv) * head_dim
+    return {"X": _normal(gen, (M, d)), "Wqkv": _normal(gen, (ncols, d), std=d ** -0.5),
+            "dQKV": _normal(gen, (M, ncols))}
+
+
+# LLaMA-7B attention input projection: 32 query and 32 key/value heads of 128, sequences of 2048.
+QKV_ROPE_7B = {"name": "rope", "M": 8192, "d": 4096, "n_q": 32, "n_kv": 32, "head_dim": 128, "seq_len": 2048,
+               "base": 10000.0}

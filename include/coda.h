@@ -246,6 +246,29 @@ coda_status coda_xent_bwd(const void* X, const void* W, const int32_t* targets, 
                           const float* dloss, void* dX, void* dW, int M, int d, int V,
                           void* ws, size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------- QKV projection with RoPE */
+
+/* QKV = X Wqkv^T with rotary position embedding applied in the GEMM's
+ * epilogue (RoPE as an elementwise transform: toolin.ai five-primitive
+ * table).  Columns are [q heads | k heads | v heads] (n_q, n_kv, n_kv heads of
+ * head_dim each); in every q and k head the pair (j, j + head_dim/2) turns by
+ * pos * base^(-2j/head_dim), pos = token row mod seq_len; v passes through.
+ * Inputs X [M,d] bf16, Wqkv [(n_q + 2 n_kv) head_dim, d] bf16.  Output QKV
+ * [M, (n_q + 2 n_kv) head_dim] bf16.  Requires d % 64 == 0, head_dim in
+ * {64, 128, 256}, seq_len >= 1, base > 1.  ws: coda_gemm_workspace_bytes(). */
+coda_status coda_qkv_rope_fwd(const void* X, const void* Wqkv, void* QKV, int M, int d, int n_q, int n_kv,
+                              int head_dim, int seq_len, float base, void* ws, size_t ws_bytes, void* stream);
+
+/* Workspace for coda_qkv_rope_bwd: status word and dPre [M, (n_q + 2 n_kv) head_dim] bf16. */
+size_t coda_qkv_rope_bwd_workspace_bytes(int M, int d, int n_q, int n_kv, int head_dim);
+
+/* Backward for the loss <dQKV, QKV>: dPre = inverse rotation of the q/k
+ * gradient (v copied), then dX = dPre Wqkv and dW = dPre^T X.
+ * Outputs dX [M,d], dW [(n_q + 2 n_kv) head_dim, d] bf16.  Same rules. */
+coda_status coda_qkv_rope_bwd(const void* dQKV, const void* X, const void* Wqkv, void* dX, void* dW, int M, int d,
+                              int n_q, int n_kv, int head_dim, int seq_len, float base,
+                              void* ws, size_t ws_bytes, void* stream);
+
 /* ---------------------------------------------------------------- unfused comparison sequence */
 
 /* The same block run operator by operator, the way a framework without
