@@ -2,6 +2,8 @@
 
 from .coda_oracle import (  # noqa: F401
     gemm,
+    mlp_block_backward,
+    mlp_block_forward,
     grg_backward_stored,
     grg_forward_stored,
     round_bf16,

@@ -61,6 +61,8 @@ __all__ = [
     "rope_rotate",
     "qkv_rope_forward",
     "qkv_rope_backward",
+    "mlp_block_forward",
+    "mlp_block_backward",
 ]
 
 
@@ -431,3 +433,44 @@ def qkv_rope_backward(dQKV, X, Wqkv, n_q: int, n_kv: int, head_dim: int, seq_len
     if store is not None:
         dpre = store(dpre)
     return {"dpre": dpre, "dX": dpre @ Wqkv, "dW": dpre.T @ X}
+
+
+# ----------------------------------------------------------------------------- full MLP block
+
+def mlp_block_forward(X, W1, R, g, W2, Wdown, eps: float, stored: bool = False, store=round_bf16) -> dict:
+    """The block followed by the down projection and its residual:
+
+      (H, r, a, b, Y) = the GEMM-Residual-RMSNorm-GEMM-SwiGLU forward
+      Out = Y Wdown^T + H               (Wdown [d, F]; the next block's residual stream)
+    The pages name residual add and SwiGLU among the epilogue transforms of
+    the same family of GEMMs (toolin.ai five-primitive table).  With
+    stored=True the GEMM-RMSNorm-GEMM part follows grg_forward_stored and the
+    down GEMM reads the stored Y and the stored H.
+    """
+    Wdown = _f64(Wdown)
+    if stored:
+        f = grg_forward_stored(X, W1, R, g, W2, eps, store)
+        out = store(f["Y"]) @ Wdown.T + f["H"]
+    else:
+        f = grg_forward(X, W1, R, g, W2, eps)
+        out = f["Y"] @ Wdown.T + f["H"]
+    return {**f, "Out": out}
+
+
+def mlp_block_backward(dOut, X, W1, R, g, W2, Wdown, eps: float, stored: bool = False, store=round_bf16,
+                       fwd: dict | None = None) -> dict:
+    """Gradients of <dOut, Out> for mlp_block_forward by the chain rule:
+      dY = dOut Wdown;  dWdown = dOut^T Y;  the residual passes dOut to H,
+      then the block's backward with upstream (dY, dH_in = dOut).
+    """
+    if fwd is None:
+        fwd = mlp_block_forward(X, W1, R, g, W2, Wdown, eps, stored, store)
+    dOut, Wdown = _f64(dOut), _f64(Wdown)
+    dY = dOut @ Wdown
+    Ys = store(fwd["Y"]) if stored else fwd["Y"]
+    dWdown = dOut.T @ Ys
+    if stored:
+        b = grg_backward_stored(dY, X, W1, R, g, W2, eps, dH_in=dOut, store=store, fwd=fwd)
+    else:
+        b = grg_backward(dY, X, W1, R, g, W2, eps, dH_in=dOut, fwd=fwd)
+    return {**b, "dY": dY, "dWdown": dWdown}

@@ -465,3 +465,43 @@ def test_qkv_rope_backward_finite_differences():
     # v columns pass through unrotated.
     f = O.qkv_rope_forward(p["X"], p["W"], nq, nkv, hd, S, 50.0)
     np.testing.assert_array_equal(f["QKV"][:, (nq + nkv) * hd:], f["pre"][:, (nq + nkv) * hd:])
+
+
+# ----------------------------------------------------------------------------- full MLP block
+
+def test_mlp_block_finite_differences():
+    rng = np.random.default_rng(22)
+    M, K, d, F, eps = 3, 5, 6, 4, 0.05
+    p = {
+        "X": rng.standard_normal((M, K)),
+        "W1": rng.standard_normal((d, K)) / np.sqrt(K),
+        "R": rng.standard_normal((M, d)),
+        "g": 1 + 0.1 * rng.standard_normal(d),
+        "W2": rng.standard_normal((2 * F, d)) / np.sqrt(d),
+        "Wdown": rng.standard_normal((d, F)) / np.sqrt(F),
+    }
+    dOut = rng.standard_normal((M, d))
+
+    def loss(q):
+        return float(np.sum(dOut * O.mlp_block_forward(q["X"], q["W1"], q["R"], q["g"], q["W2"], q["Wdown"],
+                                                        eps)["Out"]))
+
+    b = O.mlp_block_backward(dOut, p["X"], p["W1"], p["R"], p["g"], p["W2"], p["Wdown"], eps)
+    grads = {"X": b["dX"], "W1": b["dW1"], "R": b["dR"], "g": b["dg"], "W2": b["dW2"], "Wdown": b["dWdown"]}
+    _fd_check(loss, p, grads, list(grads))
+
+
+def test_mlp_block_stored_reduces_to_textbook():
+    rng = np.random.default_rng(23)
+    M, K, d, F, eps = 6, 8, 12, 10, 1e-5
+    X, R = rng.standard_normal((M, K)), rng.standard_normal((M, d))
+    W1, W2 = rng.standard_normal((d, K)) / 3, rng.standard_normal((2 * F, d)) / 3
+    Wd, g = rng.standard_normal((d, F)) / 3, 1 + 0.1 * rng.standard_normal(d)
+    dOut = rng.standard_normal((M, d))
+    f0 = O.mlp_block_forward(X, W1, R, g, W2, Wd, eps)
+    f1 = O.mlp_block_forward(X, W1, R, g, W2, Wd, eps, stored=True, store=_ident)
+    np.testing.assert_allclose(f1["Out"], f0["Out"], rtol=1e-12, atol=1e-12)
+    b0 = O.mlp_block_backward(dOut, X, W1, R, g, W2, Wd, eps, fwd=f0)
+    b1 = O.mlp_block_backward(dOut, X, W1, R, g, W2, Wd, eps, stored=True, store=_ident, fwd=f1)
+    for k in ("dX", "dR", "dW1", "dW2", "dg", "dWdown"):
+        np.testing.assert_allclose(b1[k], b0[k], rtol=1e-11, atol=1e-11, err_msg=k)
