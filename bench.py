@@ -39,6 +39,7 @@ WORKLOADS = {
     "70B": ("grg", dict(M=4096, K=8192, d=8192, F=28672, eps=1e-5), True),
     "swiglu": ("swiglu", dict(M=16384, d=4096, F=14336), True),
     "xent": ("xent", dict(M=8192, d=4096, V=128256), True),
+    "block7B": ("block", dict(M=8192, K=4096, d=4096, F=11008, eps=1e-6), True),
     "rope": ("rope", dict(M=8192, d=4096, n_q=32, n_kv=32, head_dim=128, seq_len=2048, base=10000.0), True),
 }
 
@@ -65,6 +66,9 @@ def _peaks():
 
 
 def _flops(kind, s, bwd):
+    if kind == "block":  # the block plus the down projection
+        fwd = 2.0 * s["M"] * s["K"] * s["d"] + 2.0 * s["M"] * s["d"] * 2 * s["F"] + 2.0 * s["M"] * s["F"] * s["d"]
+        return fwd * (3.0 if bwd else 1.0)
     if kind == "rope":
         return 2.0 * s["M"] * s["d"] * (s["n_q"] + 2 * s["n_kv"]) * s["head_dim"] * (3.0 if bwd else 1.0)
     if kind == "xent":  # logits GEMM forward, dX and dW backward (the backward's recompute is not counted)
@@ -83,6 +87,8 @@ def _describe(name, kind, s, bwd):
         what = "LM-head cross-entropy fwd+bwd (LLaMA-3 vocabulary)"
     elif kind == "rope":
         what = "QKV projection with RoPE epilogue fwd+bwd (LLaMA-7B attention)"
+    elif kind == "block":
+        what = f"full MLP block (GEMM-Residual-RMSNorm-GEMM-SwiGLU + down projection + residual) {name} fwd+bwd"
     else:
         what = "SwiGLU MLP fwd+bwd"
     return {"workload": what, **s, "global_batch": s["M"]}
@@ -105,6 +111,13 @@ def _oracle_step(kind, s, bwd, inputs, rows):
     """The fp64 oracle over the first `rows` tokens of the workload (forward row-local,
     weight gradients summed over those rows only)."""
     from oracle import coda_oracle as O
+    if kind == "block":
+        X, R, dOut = inputs["X"][:rows], inputs["R"][:rows], inputs["dOut"][:rows]
+        fwd = O.mlp_block_forward(X, inputs["W1"], R, inputs["g"], inputs["W2"], inputs["Wdown"], s["eps"])
+        if bwd:
+            O.mlp_block_backward(dOut, X, inputs["W1"], R, inputs["g"], inputs["W2"], inputs["Wdown"], s["eps"],
+                                 fwd=fwd)
+        return
     if kind == "rope":
         X = inputs["X"][:rows]
         a = (s["n_q"], s["n_kv"], s["head_dim"], s["seq_len"], s["base"])
@@ -138,6 +151,8 @@ def _oracle_inputs(kind, s):
         t = synth.grg_inputs(s["M"], s["K"], s["d"], s["F"], seed=0)
     elif kind == "rope":
         t = synth.qkv_inputs(s["M"], s["d"], s["n_q"], s["n_kv"], s["head_dim"], seed=0)
+    elif kind == "block":
+        t = synth.mlp_block_inputs(s["M"], s["K"], s["d"], s["F"], seed=0)
     elif kind == "xent":
         t = synth.xent_inputs(s["M"], s["d"], s["V"], seed=0)
         out = {k: v.to(torch.float64).numpy() for k, v in t.items() if k != "targets"}
@@ -287,6 +302,8 @@ def _setup(kind, s, bwd, device):
         host = synth.xent_inputs(s["M"], s["d"], s["V"], seed=0)
     elif kind == "rope":
         host = synth.qkv_inputs(s["M"], s["d"], s["n_q"], s["n_kv"], s["head_dim"], seed=0)
+    elif kind == "block":
+        host = synth.mlp_block_inputs(s["M"], s["K"], s["d"], s["F"], seed=0)
     else:
         host = synth.swiglu_inputs(s["M"], s["d"], s["F"], seed=0)
     dev = {k: v.to(device) for k, v in host.items()}
@@ -325,6 +342,20 @@ def _make_step(kind, s, bwd, dev):
         outs = {**fo, **bo}
         keys = ["Y", "dX", "dR", "dW1", "dW2", "dg"] if bwd else ["Y", "H", "r"]
         return step, outs, (10 if bwd else 4), keys, ws
+    if kind == "block":
+        K, d, F = s["K"], s["d"], s["F"]
+        ws = B.Workspace(max(lib.coda_mlp_block_fwd_workspace_bytes(M, K, d, F),
+                             lib.coda_mlp_block_bwd_workspace_bytes(M, K, d, F)), dev["X"].device)
+        fo = B.mlp_block_fwd(dev["X"], dev["W1"], dev["R"], dev["g"], dev["W2"], dev["Wdown"], s["eps"], ws=ws)
+        bo = B.mlp_block_bwd(dev["dOut"], dev["X"], dev["W1"], fo["H"], fo["r"], fo["AB"], fo["Y"], dev["g"],
+                             dev["W2"], dev["Wdown"], ws=ws)
+
+        def bstep():
+            B.mlp_block_fwd(dev["X"], dev["W1"], dev["R"], dev["g"], dev["W2"], dev["Wdown"], s["eps"], out=fo, ws=ws)
+            B.mlp_block_bwd(dev["dOut"], dev["X"], dev["W1"], fo["H"], fo["r"], fo["AB"], fo["Y"], dev["g"],
+                            dev["W2"], dev["Wdown"], out=bo, ws=ws)
+
+        return bstep, {**fo, **bo}, 13, ["Out", "dX", "dR", "dW1", "dW2", "dg", "dWdown"], ws
     if kind == "rope":
         a = (s["n_q"], s["n_kv"], s["head_dim"], s["seq_len"], s["base"])
         ws = B.Workspace(lib.coda_qkv_rope_bwd_workspace_bytes(M, s["d"], s["n_q"], s["n_kv"], s["head_dim"]),
@@ -422,7 +453,7 @@ def _dominant_kernel(kind, s, dev, outs, reps=20):
         e1.record(st)
         torch.cuda.synchronize()
         return "xent_fwd (logits GEMM + online-LSE epilogue, row reduce)", e0.elapsed_time(e1) / reps, 2.0 * M * d * V
-    if kind == "grg":
+    if kind in ("grg", "block"):
         A, W, r = outs["H"], dev["W2"], outs["r"]  # same shape and work as GEMM2 on W2g
         K = s["d"]
     else:

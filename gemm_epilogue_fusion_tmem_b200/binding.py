@@ -76,6 +76,10 @@ def library() -> ctypes.CDLL:
             "coda_qkv_rope_fwd": (I, [P, P, P, I, I, I, I, I, I, F, P, S, P]),
             "coda_qkv_rope_bwd_workspace_bytes": (S, [I, I, I, I, I]),
             "coda_qkv_rope_bwd": (I, [P, P, P, P, P, I, I, I, I, I, I, F, P, S, P]),
+            "coda_mlp_block_fwd_workspace_bytes": (S, [I, I, I, I]),
+            "coda_mlp_block_fwd": (I, [P] * 11 + [I, I, I, I, F, P, S, P]),
+            "coda_mlp_block_bwd_workspace_bytes": (S, [I, I, I, I]),
+            "coda_mlp_block_bwd": (I, [P] * 16 + [I, I, I, I, P, S, P]),
             "coda_grg_fwd_unfused_workspace_bytes": (S, [I, I, I, I]),
             "coda_grg_fwd_unfused": (I, [P] * 10 + [I, I, I, I, F, P, S, P]),
             "coda_grg_bwd_unfused_workspace_bytes": (S, [I, I, I, I]),
@@ -467,4 +471,53 @@ def qkv_rope_bwd(dQKV, X, Wqkv, n_q: int, n_kv: int, head_dim: int, seq_len: int
     ws = ws or workspace(lib.coda_qkv_rope_bwd_workspace_bytes(M, d, n_q, n_kv, head_dim), X.device)
     _check(lib.coda_qkv_rope_bwd(_ptr(dQKV), _ptr(X), _ptr(Wqkv), _ptr(o["dX"]), _ptr(o["dW"]), M, d, n_q, n_kv,
                                  head_dim, seq_len, float(base), ws.ptr(), ws.nbytes, _stream()), "coda_qkv_rope_bwd")
+    return o
+
+
+# ------------------------------------------------------------------ full MLP block
+
+def mlp_block_fwd(X, W1, R, g, W2, Wdown, eps: float, out: dict | None = None, ws: Workspace | None = None) -> dict:
+    """Block forward plus the down projection with the residual epilogue; returns H, r, Y, AB, Out."""
+    lib = library()
+    M, K = X.shape
+    d = W1.shape[0]
+    N = W2.shape[0]
+    F = N // 2
+    _req(X, "X"), _req(W1, "W1", shape=(d, K)), _req(R, "R", shape=(M, d)), _req(g, "g", shape=(d,))
+    _req(W2, "W2", shape=(N, d)), _req(Wdown, "Wdown", shape=(d, F))
+    o = dict(out or {})
+    for k, shape, dt in (("H", (M, d), torch.bfloat16), ("r", (M,), torch.float32), ("Y", (M, F), torch.bfloat16),
+                         ("AB", (M, N), torch.bfloat16), ("Out", (M, d), torch.bfloat16)):
+        if k not in o:
+            o[k] = torch.empty(*shape, dtype=dt, device=X.device)
+        _req(o[k], k, dt, shape)
+    ws = ws or workspace(lib.coda_mlp_block_fwd_workspace_bytes(M, K, d, F), X.device)
+    _check(lib.coda_mlp_block_fwd(_ptr(X), _ptr(W1), _ptr(R), _ptr(g), _ptr(W2), _ptr(Wdown), _ptr(o["H"]),
+                                  _ptr(o["r"]), _ptr(o["Y"]), _ptr(o["AB"]), _ptr(o["Out"]), M, K, d, F, float(eps),
+                                  ws.ptr(), ws.nbytes, _stream()), "coda_mlp_block_fwd")
+    return o
+
+
+def mlp_block_bwd(dOut, X, W1, H, r, AB, Y, g, W2, Wdown, out: dict | None = None,
+                  ws: Workspace | None = None) -> dict:
+    """Backward of the full block; returns dX, dR, dW1, dW2, dg, dWdown."""
+    lib = library()
+    M, K = X.shape
+    d = W1.shape[0]
+    N = W2.shape[0]
+    F = N // 2
+    _req(dOut, "dOut", shape=(M, d)), _req(X, "X"), _req(W1, "W1", shape=(d, K)), _req(H, "H", shape=(M, d))
+    _req(r, "r", torch.float32, (M,)), _req(AB, "AB", shape=(M, N)), _req(Y, "Y", shape=(M, F))
+    _req(g, "g", shape=(d,)), _req(W2, "W2", shape=(N, d)), _req(Wdown, "Wdown", shape=(d, F))
+    o = dict(out or {})
+    for k, shape, dt in (("dX", (M, K), torch.bfloat16), ("dR", (M, d), torch.bfloat16),
+                         ("dW1", (d, K), torch.bfloat16), ("dW2", (N, d), torch.bfloat16),
+                         ("dg", (d,), torch.float32), ("dWdown", (d, F), torch.bfloat16)):
+        if k not in o:
+            o[k] = torch.empty(*shape, dtype=dt, device=X.device)
+    ws = ws or workspace(lib.coda_mlp_block_bwd_workspace_bytes(M, K, d, F), X.device)
+    _check(lib.coda_mlp_block_bwd(_ptr(dOut), _ptr(X), _ptr(W1), _ptr(H), _ptr(r), _ptr(AB), _ptr(Y), _ptr(g),
+                                  _ptr(W2), _ptr(Wdown), _ptr(o["dX"]), _ptr(o["dR"]), _ptr(o["dW1"]), _ptr(o["dW2"]),
+                                  _ptr(o["dg"]), _ptr(o["dWdown"]), M, K, d, F, ws.ptr(), ws.nbytes, _stream()),
+           "coda_mlp_block_bwd")
     return o

@@ -528,6 +528,40 @@ BwdWs bwd_ws(int M, int d, int N) {
 }
 }  // namespace
 
+namespace {
+// The backward after dA' = r [da | db] and c are known:
+//   dn GEMM: dR = dH = g * (dA' W2) - c * H (+ dH_in), with dg column partials;
+//   dg column reduce;  dW2 = g * (dA'^T H);  dX = dH W1;  dW1 = dH^T X.
+coda_status grg_bwd_tail(const __nv_bfloat16* dAp, const float* cvec, float* Pg, const void* dH_in_or_null,
+                         const void* X, const void* W1, const void* H, const void* g, const void* W2, void* dX,
+                         void* dR, void* dW1, void* dW2, float* dg, int M, int K, int d, int N, void* ws,
+                         cudaStream_t s, bool pair) {
+  {
+    CUtensorMap ta, tb;
+    if (!make_operand_map(&ta, dAp, M, N, false, BM) || !make_operand_map(&tb, W2, d, N, true, BN))
+      return CODA_ERR_CUDA;
+    GemmParams p = base_params(M, d, N, BN, ws, pair);
+    p.group_m = pick_group(M, d, N, p.num_m_tiles, p.num_n_tiles, pair, num_sms());
+    p.out = bf(dR);
+    p.ldo = d;
+    p.in0 = cbf(H);
+    p.ld_in0 = d;
+    p.in1 = cbf(dH_in_or_null);
+    p.colvec = cbf(g);
+    p.rowvec = cvec;
+    p.part = Pg;
+    p.ld_part = d;
+    CODA_TRY((launch_gemm<EPI_DN, false, true>(ta, tb, p, s, pair)));
+  }
+  // One partial row per 32 output rows of every (possibly partial) row tile.
+  CODA_TRY(launch_status(launch_ex(col_reduce_kernel, dim3(cdiv(d, 32)), dim3(COLRED_THREADS), 0, s, 1,
+                                   (const float*)Pg, cdiv(M, tile_m(pair)) * tile_m(pair) / 32, d, dg)));
+  CODA_TRY(gemm_store(dAp, H, dW2, N, d, M, true, true, g, ws, s));
+  CODA_TRY(gemm_store(dR, W1, dX, M, K, d, false, true, nullptr, ws, s));
+  return gemm_store(dR, X, dW1, d, K, M, true, true, nullptr, ws, s);
+}
+}  // namespace
+
 size_t coda_grg_bwd_workspace_bytes(int M, int K, int d, int N) {
   (void)K;
   if (M < 1 || d < 1 || N < 1) return kStatusBytes;
@@ -559,33 +593,7 @@ coda_status coda_grg_bwd(const void* dY, const void* dH_in_or_null, const void* 
   // SwiGLU backward + RMSNorm row statistic.
   CODA_TRY(launch_status(launch_ex(swiglu_bwd_rowstat_kernel, dim3(M), dim3(ROWSTAT_THREADS), 0, s, 1, cbf(dY),
                                    cbf(AB), r, dAp, cvec, F, 1.0f / (float)d)));
-  // dn GEMM: dR = g * (dA' W2) - c * H (+ dH_in), with dg column partials.
-  {
-    CUtensorMap ta, tb;
-    if (!make_operand_map(&ta, dAp, M, N, false, BM) || !make_operand_map(&tb, W2, d, N, true, BN))
-      return CODA_ERR_CUDA;
-    GemmParams p = base_params(M, d, N, BN, ws, pair);
-    p.group_m = pick_group(M, d, N, p.num_m_tiles, p.num_n_tiles, pair, num_sms());
-    p.out = bf(dR);
-    p.ldo = d;
-    p.in0 = cbf(H);
-    p.ld_in0 = d;
-    p.in1 = cbf(dH_in_or_null);
-    p.colvec = cbf(g);
-    p.rowvec = cvec;
-    p.part = Pg;
-    p.ld_part = d;
-    CODA_TRY((launch_gemm<EPI_DN, false, true>(ta, tb, p, s, pair)));
-  }
-  // One partial row per 32 output rows of every (possibly partial) row tile.
-  CODA_TRY(launch_status(launch_ex(col_reduce_kernel, dim3(cdiv(d, 32)), dim3(COLRED_THREADS), 0, s, 1, (const float*)Pg,
-                                   cdiv(M, tile_m(pair)) * tile_m(pair) / 32, d, dg)));
-  // dW2 = g * (dA'^T H).
-  CODA_TRY(gemm_store(dAp, H, dW2, N, d, M, true, true, g, ws, s));
-  // dX = dH W1;  dW1 = dH^T X.
-  CODA_TRY(gemm_store(dR, W1, dX, M, K, d, false, true, nullptr, ws, s));
-  CODA_TRY(gemm_store(dR, X, dW1, d, K, M, true, true, nullptr, ws, s));
-  return CODA_OK;
+  return grg_bwd_tail(dAp, cvec, Pg, dH_in_or_null, X, W1, H, g, W2, dX, dR, dW1, dW2, dg, M, K, d, N, ws, s, pair);
 }
 
 // ------------------------------------------------------------------ SwiGLU MLP
@@ -748,6 +756,108 @@ coda_status coda_xent_bwd(const void* X, const void* W, const int32_t* targets, 
   }
   CODA_TRY(gemm_store(dlogits, W, dX, M, d, V, false, true, nullptr, ws, s));
   return gemm_store(dlogits, X, dW, V, d, M, true, true, nullptr, ws, s);
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------ full MLP block
+
+extern "C" {
+
+size_t coda_mlp_block_fwd_workspace_bytes(int M, int K, int d, int F) {
+  return coda_grg_fwd_workspace_bytes(M, K, d, 2 * F, 0);
+}
+
+coda_status coda_mlp_block_fwd(const void* X, const void* W1, const void* R, const void* g, const void* W2,
+                               const void* Wdown, void* H, float* r, void* Y, void* AB, void* Out, int M, int K,
+                               int d, int F, float eps, void* ws, size_t ws_bytes, void* stream) {
+  if (!Wdown || !Out || !AB) return CODA_ERR_INVALID_ARG;
+  if (!aligned16(Wdown) || !aligned16(Out)) return CODA_ERR_MISALIGNED;
+  // Validates every other argument and runs the block's forward.
+  CODA_TRY(coda_grg_fwd(X, W1, R, g, W2, nullptr, H, r, Y, AB, M, K, d, 2 * F, eps, ws, ws_bytes, stream));
+  // Down projection with the residual in its epilogue: Out = Y Wdown^T + H.
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool pair = use_pair();
+  CUtensorMap ta, tb;
+  if (!make_operand_map(&ta, Y, M, F, false, BM) || !make_operand_map(&tb, Wdown, d, F, false, pair ? BN / 2 : BN))
+    return CODA_ERR_CUDA;
+  GemmParams p = base_params(M, d, F, BN, ws, pair);
+  p.group_m = pick_group(M, d, F, p.num_m_tiles, p.num_n_tiles, pair, num_sms());
+  p.out = bf(Out);
+  p.ldo = d;
+  p.in0 = cbf(H);
+  p.ld_in0 = d;
+  return launch_gemm<EPI_RESID_RMS, false, false>(ta, tb, p, s, pair);
+}
+
+namespace {
+struct BlockBwdWs {
+  BwdWs b;
+  size_t pc_off, total;
+  int T;
+};
+BlockBwdWs block_bwd_ws(int M, int d, int F) {
+  BlockBwdWs w;
+  w.b = bwd_ws(M, d, 2 * F);
+  w.T = cdiv(F, BN);
+  w.pc_off = w.b.total;
+  w.total = align_up(w.pc_off + (size_t)M * w.T * 4, 256);
+  return w;
+}
+}  // namespace
+
+size_t coda_mlp_block_bwd_workspace_bytes(int M, int K, int d, int F) {
+  (void)K;
+  if (M < 1 || d < 1 || F < 1) return kStatusBytes;
+  return block_bwd_ws(M, d, F).total;
+}
+
+coda_status coda_mlp_block_bwd(const void* dOut, const void* X, const void* W1, const void* H, const float* r,
+                               const void* AB, const void* Y, const void* g, const void* W2, const void* Wdown,
+                               void* dX, void* dR, void* dW1, void* dW2, float* dg, void* dWdown, int M, int K, int d,
+                               int F, void* ws, size_t ws_bytes, void* stream) {
+  if (!dOut || !X || !W1 || !H || !r || !AB || !Y || !g || !W2 || !Wdown || !dX || !dR || !dW1 || !dW2 || !dg ||
+      !dWdown || !ws)
+    return CODA_ERR_INVALID_ARG;
+  CODA_TRY(check_grg_shapes(M, K, d, 2 * F));
+  const void* ptrs[] = {dOut, X, W1, H, r, AB, Y, g, W2, Wdown, dX, dR, dW1, dW2, dg, dWdown, ws};
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return CODA_ERR_MISALIGNED;
+  const BlockBwdWs w = block_bwd_ws(M, d, F);
+  if (ws_bytes < w.total) return CODA_ERR_WORKSPACE_TOO_SMALL;
+  int dev;
+  CODA_TRY(current_device(dev));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  __nv_bfloat16* dAp = reinterpret_cast<__nv_bfloat16*>(wsb + w.b.dap_off);
+  float* cvec = reinterpret_cast<float*>(wsb + w.b.c_off);
+  float* Pg = reinterpret_cast<float*>(wsb + w.b.pg_off);
+  float* Pc = reinterpret_cast<float*>(wsb + w.pc_off);
+  const int N = 2 * F;
+  const bool pair = use_pair();
+  // Down-projection dgrad with the SwiGLU backward, the r scale and the row
+  // partials of c in its epilogue: dY never reaches HBM.
+  {
+    CUtensorMap ta, tb;
+    if (!make_operand_map(&ta, dOut, M, d, false, BM) || !make_operand_map(&tb, Wdown, F, d, true, BN))
+      return CODA_ERR_CUDA;
+    GemmParams p = base_params(M, F, d, BN, ws, pair);
+    p.group_m = pick_group(M, F, d, p.num_m_tiles, p.num_n_tiles, pair, num_sms());
+    p.split = F;
+    p.out = dAp;
+    p.ldo = N;
+    p.in0 = cbf(AB);
+    p.ld_in0 = N;
+    p.rowvec = r;
+    p.part = Pc;
+    p.ld_part = w.T;
+    CODA_TRY((launch_gemm<EPI_SWIGLU_BWD, false, true>(ta, tb, p, s, pair)));
+  }
+  CODA_TRY(launch_status(launch_ex(rowcoef_reduce_kernel, dim3(cdiv(M, 256)), dim3(256), 0, s, 1, (const float*)Pc,
+                                   w.T, r, cvec, M, 1.0f / (float)d)));
+  CODA_TRY(gemm_store(dOut, Y, dWdown, d, F, M, true, true, nullptr, ws, s));
+  // The residual Out = ... + H sends dOut straight into dH.
+  return grg_bwd_tail(dAp, cvec, Pg, dOut, X, W1, H, g, W2, dX, dR, dW1, dW2, dg, M, K, d, N, ws, s, pair);
 }
 
 }  // extern "C"

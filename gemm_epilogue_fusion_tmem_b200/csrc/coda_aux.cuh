@@ -42,6 +42,19 @@ __global__ void rms_rowreduce_kernel(const float* __restrict__ P, int T, float* 
   r[i] = rsqrtf(fmaf(s, inv_d, eps));
 }
 
+// c_i = (r_i^2 / d) sum_t Pc[i, t]: the RMSNorm backward's row coefficient
+// from the per-tile partials of the down-projection dgrad's epilogue.
+__global__ void rowcoef_reduce_kernel(const float* __restrict__ Pc, int T, const float* __restrict__ r,
+                                      float* __restrict__ c, int M, float inv_d) {
+  griddep_wait();
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= M) return;
+  const float* row = Pc + (size_t)i * T;
+  float s = 0.f;
+  for (int t = 0; t < T; ++t) s += row[t];
+  c[i] = r[i] * r[i] * inv_d * s;
+}
+
 template <int THREADS>
 __device__ __forceinline__ float block_sum(float v, float* scratch) {
 #pragma unroll

@@ -37,7 +37,7 @@ enum Epi : int {
   EPI_RESID_RMS = 1,   // H = bf16(acc + R); P[row, ntile] = sum bf16(H)^2; optional Hg = bf16(H*g)
   EPI_SWIGLU = 2,      // a = r*acc_gate, b = r*acc_up; Y = silu(a)*b; AB = [a|b]
   EPI_DN = 3,          // dH = g*acc - c*H (+dH_in); column partials of acc*H
-  EPI_SWIGLU_BWD = 4,  // dY = acc; da, db from a, b; dA = [da|db]
+  EPI_SWIGLU_BWD = 4,  // dY = acc; da, db from a, b; dA = [da|db] (optionally r-scaled, with c partials)
   EPI_XENT = 5,        // logits tile: per-row online (max, sum exp) partials + the target logit
   EPI_XENT_BWD = 6,    // dlogits = dloss_i (exp(logit - lse_i) - [j == t_i]), stored bf16
   EPI_ROPE = 7,        // QKV tile: rotate the q/k heads' (j, j + hd/2) pairs by pos * base^(-2j/hd)
@@ -194,7 +194,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbas
         if (rv) store32_bf16(p.out2 + (size_t)row * p.ldo + n0 + c, g);
       }
     }
-    if (rv) p.part[(size_t)row * p.ld_part + n_blk] = ss;
+    if (rv && p.part != nullptr) p.part[(size_t)row * p.ld_part + n_blk] = ss;
   } else if constexpr (EPI == EPI_SWIGLU) {
     constexpr int HALF = BN / 2;
     const int n0 = n_blk * HALF;
@@ -327,7 +327,12 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbas
       }
     }
   } else if constexpr (EPI == EPI_SWIGLU_BWD) {
+    // dA = [da | db] from dY = acc and the saved a, b.  With a row scale r
+    // (rowvec) the stored operand is r_i [da | db] and the tile also emits the
+    // row partial sum_c (da a + db b) of the RMSNorm backward's coefficient.
     const int n0 = n_blk * BN;
+    const float rr = (p.rowvec != nullptr) ? (rv ? p.rowvec[row] : 0.f) : 1.f;
+    float cpart = 0.f;
 #pragma unroll 1
     for (int c = 0; c < BN; c += 32) {
       if (n0 + c >= p.N) break;
@@ -342,8 +347,10 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbas
         const float s = sigmoid_f(a[i]);
         const float da = dy[i] * b[i] * s * (1.f + a[i] * (1.f - s));
         const float db = dy[i] * a[i] * s;
-        a[i] = da;
-        b[i] = db;
+        cpart = fmaf(da, a[i], cpart);
+        cpart = fmaf(db, b[i], cpart);
+        a[i] = da * rr;
+        b[i] = db * rr;
       }
       if (rv) {
         __nv_bfloat16* dst = p.out + (size_t)row * p.ldo + n0 + c;
@@ -351,6 +358,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbas
         store32_bf16(dst + p.split, b);
       }
     }
+    if (rv && p.part != nullptr) p.part[(size_t)row * p.ld_part + n_blk] = cpart;
   }
 }
 

@@ -130,3 +130,15 @@ def qkv_inputs(M: int, d: int, n_q: int, n_kv: int, head_dim: int, seed: int = 0
 # LLaMA-7B attention input projection: 32 query and 32 key/value heads of 128, sequences of 2048.
 QKV_ROPE_7B = {"name": "rope", "M": 8192, "d": 4096, "n_q": 32, "n_kv": 32, "head_dim": 128, "seq_len": 2048,
                "base": 10000.0}
+
+
+def mlp_block_inputs(M: int, K: int, d: int, F: int, seed: int = 0) -> dict:
+    """Full MLP block inputs: those of grg_inputs (X, R, W1, W2, g, dY drawn first, in that
+    order) then Wdown ~ N(0, 1/F) and dOut ~ N(0, 1); dY is dropped (the block's upstream
+    gradient is dOut)."""
+    t = grg_inputs(M, K, d, F, seed=seed)
+    gen = torch.Generator().manual_seed(seed + 7919)
+    t.pop("dY")
+    t["Wdown"] = _normal(gen, (d, F), std=F ** -0.5)
+    t["dOut"] = _normal(gen, (M, d))
+    return t

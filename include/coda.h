@@ -216,6 +216,40 @@ coda_status coda_swiglu_bwd(const void* dOut, const void* X, const void* Wgu, co
                             void* dX, void* dWgu, void* dWdown,
                             int M, int d, int F, void* ws, size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------- full MLP block */
+
+/* Workspace for coda_mlp_block_fwd (that of coda_grg_fwd without a pre-folded weight). */
+size_t coda_mlp_block_fwd_workspace_bytes(int M, int K, int d, int F);
+
+/* The block followed by the down projection, whose epilogue adds the residual
+ * for the next block (residual add as an elementwise epilogue transform,
+ * toolin.ai five-primitive table):
+ *   coda_grg_fwd (H, r, Y, AB);  Out = Y Wdown^T + H  (bf16 [M, d]).
+ * Inputs as coda_grg_fwd (N = 2F) plus Wdown [d, F] bf16; AB is required. */
+coda_status coda_mlp_block_fwd(const void* X, const void* W1, const void* R, const void* g, const void* W2,
+                               const void* Wdown, void* H, float* r, void* Y, void* AB, void* Out,
+                               int M, int K, int d, int F, float eps, void* ws, size_t ws_bytes, void* stream);
+
+/* Workspace for coda_mlp_block_bwd: that of coda_grg_bwd plus the row
+ * partials of c [M, ceil(F/256)] fp32. */
+size_t coda_mlp_block_bwd_workspace_bytes(int M, int K, int d, int F);
+
+/* Backward of <dOut, Out> for coda_mlp_block_fwd.  The down projection's
+ * dgrad GEMM carries the SwiGLU backward in its epilogue, so dY never reaches
+ * HBM: dY = dOut Wdown (fp32 accumulator); da, db from the saved a, b; the
+ * stored operand dA' = bf16(r_i [da | db]) and the row partials of
+ * c_i = (r_i^2/d) sum_c (da a + db b) come out of the same epilogue (the
+ * block-local backward of kucoin (ru) «В «Финале» спрятаны сокровища»).  Then
+ * dWdown = dOut^T Y, and the block's dn GEMM (with dH_in = dOut from the
+ * residual), dg, dW2, dX, dW1 as in coda_grg_bwd.
+ * Inputs dOut [M,d], and X, W1, H, r, AB, Y, g, W2, Wdown as saved by the
+ * forward.  Outputs dX [M,K], dR [M,d], dW1 [d,K], dW2 [2F,d], dg [d] fp32,
+ * dWdown [d,F] (bf16 unless stated).  Shape rules of coda_grg_fwd. */
+coda_status coda_mlp_block_bwd(const void* dOut, const void* X, const void* W1, const void* H, const float* r,
+                               const void* AB, const void* Y, const void* g, const void* W2, const void* Wdown,
+                               void* dX, void* dR, void* dW1, void* dW2, float* dg, void* dWdown,
+                               int M, int K, int d, int F, void* ws, size_t ws_bytes, void* stream);
+
 /* ---------------------------------------------------------------- cross-entropy on the LM head */
 
 /* Workspace for coda_xent_fwd: status word, per-tile (max, sum exp) partials

@@ -108,3 +108,26 @@ def test_swiglu_full_size(cuda_lib):
         assert_tol(gpu[k], fs[k], f"swiglu {k}")
     for k in ("dX", "dWgu", "dWdown"):
         assert_tol(gpu[k], bs[k], f"swiglu {k}", outlier_frac=BWD_OUTLIER_FRAC)
+
+
+def test_mlp_block_full_size(cuda_lib):
+    """The full MLP block at the 7B shape (M=8192, K=d=4096, F=11008), fwd+bwd."""
+    from tests.parity import assert_tol as _tol
+    M, K, d, F, eps = 8192, 4096, 4096, 11008, 1e-6
+    t = synth.mlp_block_inputs(M, K, d, F, seed=0)
+    td = {k: v.cuda() for k, v in t.items()}
+    o = cuda_lib.mlp_block_fwd(td["X"], td["W1"], td["R"], td["g"], td["W2"], td["Wdown"], eps)
+    b = cuda_lib.mlp_block_bwd(td["dOut"], td["X"], td["W1"], o["H"], o["r"], o["AB"], o["Y"], td["g"], td["W2"],
+                               td["Wdown"])
+    torch.cuda.synchronize()
+    gf = {k: f64(o[k]) for k in ("Y", "Out")}
+    gb = {k: f64(v) for k, v in b.items()}
+    del o, b, td
+    torch.cuda.empty_cache()
+    X, W1, R, g, W2, Wd, dOut = (f64(t[k]) for k in ("X", "W1", "R", "g", "W2", "Wdown", "dOut"))
+    fs = O.mlp_block_forward(X, W1, R, g, W2, Wd, eps, stored=True)
+    for k, v in gf.items():
+        _tol(v, fs[k], f"block 7B {k}")
+    bs = O.mlp_block_backward(dOut, X, W1, R, g, W2, Wd, eps, stored=True, fwd=fs)
+    for k in ("dX", "dR", "dW1", "dW2", "dg", "dWdown"):
+        _tol(gb[k], bs[k], f"block 7B {k}", outlier_frac=BWD_OUTLIER_FRAC)

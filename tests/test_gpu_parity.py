@@ -221,3 +221,19 @@ def test_grg_forward_activation_gain(cuda_lib, M, K, d, F, eps):
     bs = O.grg_backward_stored(dY, X, W1, R, g, W2, eps, fwd=fs)
     for k in ("dX", "dR", "dW1", "dW2", "dg"):
         assert_tol(b[k], bs[k], f"{tag} bwd {k}", outlier_frac=BWD_OUTLIER_FRAC)
+
+
+def test_run_to_run_bit_reproducible(cuda_lib):
+    """Partials + fixed-order reduces (no atomics): two runs give identical bits."""
+    M, K, d, F, eps = 2048, 1024, 1024, 2816, 1e-6
+    t = synth.grg_inputs(M, K, d, F, seed=9, dH_in=True)
+    td = _cuda(t)
+    outs = []
+    for _ in range(2):
+        o = cuda_lib.grg_fwd(td["X"], td["W1"], td["R"], td["g"], td["W2"], eps)
+        b = cuda_lib.grg_bwd(td["dY"], td["X"], td["W1"], o["H"], o["r"], o["AB"], td["g"], td["W2"],
+                             dH_in=td["dH_in"])
+        torch.cuda.synchronize()
+        outs.append({k: v.clone() for k, v in {**o, **b}.items()})
+    for k in outs[0]:
+        assert torch.equal(outs[0][k], outs[1][k]), f"{k} differs between runs"
