@@ -55,6 +55,7 @@ def library() -> ctypes.CDLL:
             "coda_status_clear": (I, [P, P]),
             "coda_status_query": (I, [P, P, ctypes.POINTER(ctypes.c_uint32)]),
             "coda_set_wait_limit_ns": (None, [ctypes.c_uint64]),
+            "coda_selftest_wait_timeout": (I, [P, ctypes.c_uint64, P]),
             "coda_gemm_workspace_bytes": (S, []),
             "coda_gemm": (I, [P, P, P, I, I, I, I, I, P, S, P]),
             "coda_fold_gain": (I, [P, P, P, I, I, P]),
@@ -167,6 +168,11 @@ def workspace(nbytes: int, device=None) -> Workspace:
 
 def set_wait_limit_ns(ns: int) -> None:
     library().coda_set_wait_limit_ns(int(ns))
+
+
+def selftest_wait_timeout(ws: Workspace, limit_ns: int) -> None:
+    """Launch the bounded-wait self-test (a wait that must time out) on the current stream."""
+    _check(library().coda_selftest_wait_timeout(ws.ptr(), int(limit_ns), _stream()), "coda_selftest_wait_timeout")
 
 
 # ------------------------------------------------------------------ entry points

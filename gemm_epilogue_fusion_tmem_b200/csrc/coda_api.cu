@@ -319,6 +319,17 @@ void coda_set_wait_limit_ns(uint64_t ns) {
   g_wait_limit_ns.store(ns);
 }
 
+coda_status coda_selftest_wait_timeout(void* ws, uint64_t limit_ns, void* stream) {
+  if (ws == nullptr) return CODA_ERR_INVALID_ARG;
+  if (!aligned16(ws)) return CODA_ERR_MISALIGNED;
+  int dev;
+  CODA_TRY(current_device(dev));
+  limit_ns = std::min<uint64_t>(std::max<uint64_t>(limit_ns, 1000ull), 60000000000ull);
+  selftest_wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<uint32_t*>(ws),
+                                                                              (unsigned long long)limit_ns);
+  return launch_status(cudaPeekAtLastError());
+}
+
 coda_status coda_status_clear(void* ws, void* stream) {
   if (ws == nullptr) return CODA_ERR_INVALID_ARG;
   return launch_status(cudaMemsetAsync(ws, 0, kStatusBytes, static_cast<cudaStream_t>(stream)));

@@ -101,7 +101,7 @@ __global__ void __launch_bounds__(ROWSTAT_THREADS)
     unpack8(ldg_nc_v4(b + 8 * v), fb);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const float s = __frcp_rn(1.0f + __expf(-fa[i]));
+      const float s = sigmoid_f(fa[i]);
       da[i] = fy[i] * fb[i] * s * (1.f + fa[i] * (1.f - s));
       db[i] = fy[i] * fa[i] * s;
       acc = fmaf(da[i], fa[i], acc);
@@ -221,6 +221,25 @@ __global__ void xent_reduce_kernel(const float2* __restrict__ part, int T, const
     lse[row] = l;
     loss[row] = l - tlogit[row];
   }
+}
+
+// Self-test of the device-side failure path: one warp waits, with the same
+// bounded wait the GEMM pipeline uses, on an mbarrier that nothing arrives on.
+// The wait gives up after limit_ns, records CODA_ERR_DEVICE_TIMEOUT and the
+// detail word in the status word, and the kernel returns normally.
+constexpr uint32_t kSelftestKernelId = 0x3F;
+__global__ void selftest_wait_timeout_kernel(uint32_t* status, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const WaitCtl ctl{&abort_flag, status, limit_ns, kSelftestKernelId};
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, ctl, 0, kWaitFull);
+  __syncthreads();
 }
 
 }  // namespace coda

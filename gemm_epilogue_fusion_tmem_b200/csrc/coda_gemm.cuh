@@ -136,7 +136,6 @@ __device__ __forceinline__ void warp_column_sums(float (&v)[32], int lane) {
   }
 }
 
-__device__ __forceinline__ float sigmoid_f(float x) { return __frcp_rn(1.0f + __expf(-x)); }
 
 // One 128-row half-tile of the epilogue: this thread owns output row `row`
 // (valid when rv), `group32` = (row - lane) / 32 indexes the per-warp partials.

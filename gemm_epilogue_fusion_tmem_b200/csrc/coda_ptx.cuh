@@ -217,6 +217,14 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   }
 }
 
+// ------------------------------------------------------------------ elementwise math
+
+// Logistic sigmoid with the fast exponential and fast division intrinsics
+// (a few ulp in fp32, far below the bf16 rounding of every stored result).
+// Large negative x: exp overflows to inf and the quotient is 0; large
+// positive x: exp underflows to 0 and the quotient is 1.
+__device__ __forceinline__ float sigmoid_f(float x) { return __fdividef(1.0f, 1.0f + __expf(-x)); }
+
 // ------------------------------------------------------------------ bf16 packing
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

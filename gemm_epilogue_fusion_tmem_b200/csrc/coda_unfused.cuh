@@ -75,7 +75,7 @@ __global__ void unf_swiglu_fwd_kernel(const __nv_bfloat16* __restrict__ A, __nv_
     unpack8(ldg_nc_v4(A + row * 2 * F + c), a);
     unpack8(ldg_nc_v4(A + row * 2 * F + F + c), b);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) a[i] = a[i] * __frcp_rn(1.0f + __expf(-a[i])) * b[i];
+    for (int i = 0; i < 8; ++i) a[i] = a[i] * sigmoid_f(a[i]) * b[i];
     stg_v4(Y + row * F + c, pack8(a));
   }
 }
@@ -95,7 +95,7 @@ __global__ void unf_swiglu_bwd_kernel(const __nv_bfloat16* __restrict__ dY, cons
     unpack8(ldg_nc_v4(A + row * 2 * F + F + c), b);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const float s = __frcp_rn(1.0f + __expf(-a[i]));
+      const float s = sigmoid_f(a[i]);
       const float da = dy[i] * b[i] * s * (1.f + a[i] * (1.f - s));
       const float db = dy[i] * a[i] * s;
       a[i] = da;

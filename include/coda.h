@@ -81,6 +81,15 @@ coda_status coda_status_query(const void* ws, void* stream, uint32_t* detail);
  * Values are clamped to [1e3, 6e10]. */
 void coda_set_wait_limit_ns(uint64_t ns);
 
+/* Self-test of the device-side failure path: a one-warp kernel waits, with
+ * the bounded wait every pipeline barrier uses, on a barrier that nothing
+ * arrives on.  After limit_ns (clamped as above) it records
+ * CODA_ERR_DEVICE_TIMEOUT and the detail word (kernel id 0x3F, role 0,
+ * reason 1) in the workspace's status word and returns; nothing faults and
+ * the context stays usable.  Read the result with coda_status_query and clear
+ * it with coda_status_clear. */
+coda_status coda_selftest_wait_timeout(void* ws, uint64_t limit_ns, void* stream);
+
 /* ---------------------------------------------------------------- building block */
 
 /* C[M,N] (bf16) = op(A) * op(B)^T with fp32 accumulation on tcgen05 tensor cores.

@@ -32,6 +32,7 @@ GEMM_CASES = [
     (1, 256, 64),
     (384, 288, 4160),
     (2048, 4096, 256),  # 256 tiles > 148 SMs: persistent loop, both TMEM accumulators
+    (136, 96, 200),     # reduction not a multiple of 64 (zero-filled tail), N < one tile
 ]
 
 
