@@ -1,0 +1,49 @@
+"""Host-side behaviour of the Python binding (CPU only, no compute call).
+
+There is no CPU path: CPU tensors, wrong dtypes and wrong shapes are refused
+before anything reaches the library's compute entry points, and every entry
+point the binding names is exported by the built library.
+"""
+
+import pytest
+import torch
+
+from gemm_epilogue_fusion_tmem_b200 import binding as B
+
+
+def _bf(*s):
+    return torch.zeros(*s, dtype=torch.bfloat16)
+
+
+def test_library_loads_and_binds_every_entry_point():
+    lib = B.library()
+    for name in ("coda_grg_fwd", "coda_grg_bwd", "coda_swiglu_fwd", "coda_swiglu_bwd", "coda_gemm",
+                 "coda_gemm_swiglu", "coda_grg_fwd_hg", "coda_xent_fwd", "coda_xent_bwd", "coda_qkv_rope_fwd",
+                 "coda_qkv_rope_bwd", "coda_mlp_block_fwd", "coda_mlp_block_bwd", "coda_grg_fwd_unfused",
+                 "coda_grg_bwd_unfused", "coda_selftest_wait_timeout"):
+        assert getattr(lib, name).restype is not None or name == "coda_set_wait_limit_ns"
+
+
+def test_cpu_tensors_are_refused():
+    X, W1, R, g, W2 = _bf(256, 512), _bf(512, 512), _bf(256, 512), _bf(512), _bf(2048, 512)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        B.grg_fwd(X, W1, R, g, W2, 1e-6)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        B.gemm(X, W1, 256, 512, 512)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        B.xent_fwd(X, _bf(1024, 512), torch.zeros(256, dtype=torch.int32))
+
+
+def test_wrong_dtype_and_shape_are_refused():
+    X = torch.zeros(4, 8)  # float32 on CPU: the device check fires first
+    with pytest.raises(ValueError):
+        B._req(X, "X")
+    with pytest.raises(TypeError):
+        B._req("not a tensor", "X")
+
+
+def test_status_strings_round_trip():
+    assert B._status_string(0) == "ok"
+    assert "timed out" in B._status_string(B.CODA_ERR_DEVICE_TIMEOUT)
+    err = B.CodaError(3, "coda_gemm")
+    assert err.status == 3 and "16-byte" in str(err)
