@@ -442,7 +442,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ---------------------------------------------------------------- producer (every CTA)
-      const uint64_t hint = l2_policy_evict_normal();
+      // Normal L2 priority for both operands: concurrent tiles of a wave reuse
+      // each other's lines, which evict-first / evict-last hints were measured to
+      // break (DRAM reads per launch more than doubled).
+      const uint64_t hint_a = l2_policy_evict_normal();
+      const uint64_t hint_b = hint_a;
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -463,38 +467,38 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
             const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
             if constexpr (!A_MN) {
-              tma_load_2d_pair(a_dst, &tmA, bar, k0, a_row, hint);
+              tma_load_2d_pair(a_dst, &tmA, bar, k0, a_row, hint_a);
             } else {
 #pragma unroll
-              for (int c = 0; c < 2; ++c) tma_load_2d_pair(a_dst + c * MN_CHUNK_BYTES, &tmA, bar, a_row + c * 64, k0, hint);
+              for (int c = 0; c < 2; ++c) tma_load_2d_pair(a_dst + c * MN_CHUNK_BYTES, &tmA, bar, a_row + c * 64, k0, hint_a);
             }
             if constexpr (EPI == EPI_SWIGLU) {
               // Leader holds the 128 gate rows, the peer the 128 up rows of these output columns.
-              tma_load_2d_pair(b_dst, &tmB, bar, k0, (rank ? p.split : 0) + n_blk * (BN / 2), hint);
+              tma_load_2d_pair(b_dst, &tmB, bar, k0, (rank ? p.split : 0) + n_blk * (BN / 2), hint_b);
             } else if constexpr (!B_MN) {
-              tma_load_2d_pair(b_dst, &tmB, bar, k0, n_blk * BN + (int)rank * 128, hint);
+              tma_load_2d_pair(b_dst, &tmB, bar, k0, n_blk * BN + (int)rank * 128, hint_b);
             } else {
 #pragma unroll
               for (int c = 0; c < 2; ++c)
-                tma_load_2d_pair(b_dst + c * MN_CHUNK_BYTES, &tmB, bar, n_blk * BN + (int)rank * 128 + c * 64, k0, hint);
+                tma_load_2d_pair(b_dst + c * MN_CHUNK_BYTES, &tmB, bar, n_blk * BN + (int)rank * 128 + c * 64, k0, hint_b);
             }
           } else {
             uint64_t* bar = &full[stage];
             mbar_arrive_expect_tx(bar, C::STAGE_BYTES);
             if constexpr (!A_MN) {
-              tma_load_2d(a_dst, &tmA, bar, k0, a_row, hint);
+              tma_load_2d(a_dst, &tmA, bar, k0, a_row, hint_a);
             } else {
 #pragma unroll
-              for (int c = 0; c < 2; ++c) tma_load_2d(a_dst + c * MN_CHUNK_BYTES, &tmA, bar, a_row + c * 64, k0, hint);
+              for (int c = 0; c < 2; ++c) tma_load_2d(a_dst + c * MN_CHUNK_BYTES, &tmA, bar, a_row + c * 64, k0, hint_a);
             }
             if constexpr (EPI == EPI_SWIGLU) {
-              tma_load_2d(b_dst, &tmB, bar, k0, n_blk * (BN / 2), hint);
-              tma_load_2d(b_dst + C::B_BYTES / 2, &tmB, bar, k0, p.split + n_blk * (BN / 2), hint);
+              tma_load_2d(b_dst, &tmB, bar, k0, n_blk * (BN / 2), hint_b);
+              tma_load_2d(b_dst + C::B_BYTES / 2, &tmB, bar, k0, p.split + n_blk * (BN / 2), hint_b);
             } else if constexpr (!B_MN) {
-              tma_load_2d(b_dst, &tmB, bar, k0, n_blk * BN, hint);
+              tma_load_2d(b_dst, &tmB, bar, k0, n_blk * BN, hint_b);
             } else {
 #pragma unroll
-              for (int c = 0; c < BN / 64; ++c) tma_load_2d(b_dst + c * MN_CHUNK_BYTES, &tmB, bar, n_blk * BN + c * 64, k0, hint);
+              for (int c = 0; c < BN / 64; ++c) tma_load_2d(b_dst + c * MN_CHUNK_BYTES, &tmB, bar, n_blk * BN + c * 64, k0, hint_b);
             }
           }
           ++issued;
