@@ -333,12 +333,18 @@ def _make_step(kind, s, bwd, dev):
                   "dW2": torch.empty(N, d, dtype=torch.bfloat16, device=dev["X"].device),
                   "dg": torch.empty(d, dtype=torch.float32, device=dev["X"].device)}
 
-        def step():
+        def fwd_only():
             B.grg_fwd(dev["X"], dev["W1"], dev["R"], dev["g"], dev["W2"], s["eps"], out=fo, ws=ws)
-            if bwd:
-                B.grg_bwd(dev["dY"], dev["X"], dev["W1"], fo["H"], fo["r"], fo["AB"], dev["g"], dev["W2"],
-                          out=bo, ws=ws)
 
+        def bwd_only():
+            B.grg_bwd(dev["dY"], dev["X"], dev["W1"], fo["H"], fo["r"], fo["AB"], dev["g"], dev["W2"], out=bo, ws=ws)
+
+        def step():
+            fwd_only()
+            if bwd:
+                bwd_only()
+
+        step.fwd, step.bwd = fwd_only, (bwd_only if bwd else None)
         outs = {**fo, **bo}
         keys = ["Y", "dX", "dR", "dW1", "dW2", "dg"] if bwd else ["Y", "H", "r"]
         return step, outs, (10 if bwd else 4), keys, ws
@@ -385,36 +391,84 @@ def _make_step(kind, s, bwd, dev):
     fo = B.swiglu_fwd(dev["X"], dev["Wgu"], dev["Wdown"], ws=ws)
     bo = B.swiglu_bwd(dev["dOut"], dev["X"], dev["Wgu"], dev["Wdown"], fo["Y"], fo["AB"], ws=ws)
 
-    def step():
+    def fwd_only():
         B.swiglu_fwd(dev["X"], dev["Wgu"], dev["Wdown"], out=fo, ws=ws)
+
+    def bwd_only():
         B.swiglu_bwd(dev["dOut"], dev["X"], dev["Wgu"], dev["Wdown"], fo["Y"], fo["AB"], out=bo, ws=ws)
 
+    def step():
+        fwd_only()
+        bwd_only()
+
+    step.fwd, step.bwd = fwd_only, bwd_only
     outs = {**fo, **bo}
     return step, outs, 6, ["Out", "dX", "dWgu", "dWdown"], ws
 
 
-def _make_unfused_step(s, bwd, dev):
-    """The same block run operator by operator (every intermediate in HBM)."""
+def _make_unfused_step(kind, s, bwd, dev):
+    """The same work run operator by operator (every intermediate in HBM)."""
     import torch
     from gemm_epilogue_fusion_tmem_b200 import binding as B
     lib = B.library()
-    M, K, d, F = s["M"], s["K"], s["d"], s["F"]
-    N = 2 * F
-    ws = B.Workspace(max(lib.coda_grg_fwd_unfused_workspace_bytes(M, K, d, N),
-                         lib.coda_grg_bwd_unfused_workspace_bytes(M, K, d, N)), dev["X"].device)
-    fo = B.grg_fwd_unfused(dev["X"], dev["W1"], dev["R"], dev["g"], dev["W2"], s["eps"], ws=ws)
-    bo = {}
-    if bwd:
-        bo = B.grg_bwd_unfused(dev["dY"], dev["X"], dev["W1"], fo["H"], fo["r"], fo["AB"], fo["U"], dev["g"],
-                               dev["W2"], ws=ws)
+    if kind == "swiglu":
+        M, d, F = s["M"], s["d"], s["F"]
+        ws = B.Workspace(lib.coda_swiglu_bwd_unfused_workspace_bytes(M, d, F), dev["X"].device)
+        fo = B.swiglu_fwd_unfused(dev["X"], dev["Wgu"], dev["Wdown"], ws=ws)
+        bo = B.swiglu_bwd_unfused(dev["dOut"], dev["X"], dev["Wgu"], dev["Wdown"], fo["Y"], fo["AB"], ws=ws)
 
-    def step():
-        B.grg_fwd_unfused(dev["X"], dev["W1"], dev["R"], dev["g"], dev["W2"], s["eps"], out=fo, ws=ws)
+        def fwd_only():
+            B.swiglu_fwd_unfused(dev["X"], dev["Wgu"], dev["Wdown"], out=fo, ws=ws)
+
+        def bwd_only():
+            B.swiglu_bwd_unfused(dev["dOut"], dev["X"], dev["Wgu"], dev["Wdown"], fo["Y"], fo["AB"], out=bo, ws=ws)
+
+        launches = 3 + 5
+    else:
+        M, K, d, F = s["M"], s["K"], s["d"], s["F"]
+        N = 2 * F
+        ws = B.Workspace(max(lib.coda_grg_fwd_unfused_workspace_bytes(M, K, d, N),
+                             lib.coda_grg_bwd_unfused_workspace_bytes(M, K, d, N)), dev["X"].device)
+        fo = B.grg_fwd_unfused(dev["X"], dev["W1"], dev["R"], dev["g"], dev["W2"], s["eps"], ws=ws)
+        bo = {}
         if bwd:
+            bo = B.grg_bwd_unfused(dev["dY"], dev["X"], dev["W1"], fo["H"], fo["r"], fo["AB"], fo["U"], dev["g"],
+                                   dev["W2"], ws=ws)
+
+        def fwd_only():
+            B.grg_fwd_unfused(dev["X"], dev["W1"], dev["R"], dev["g"], dev["W2"], s["eps"], out=fo, ws=ws)
+
+        def bwd_only():
             B.grg_bwd_unfused(dev["dY"], dev["X"], dev["W1"], fo["H"], fo["r"], fo["AB"], fo["U"], dev["g"],
                               dev["W2"], out=bo, ws=ws)
 
-    return step, (13 if bwd else 5), ws
+        launches = 5 + (8 if bwd else 0)
+
+    def step():
+        fwd_only()
+        if bwd:
+            bwd_only()
+
+    step.fwd, step.bwd = fwd_only, (bwd_only if bwd else None)
+    return step, launches, ws
+
+
+def _time_loop(fn, steps, warmup, device, world, barrier):
+    """Device time of `steps` calls of fn (CUDA events on the current stream), max over ranks."""
+    import torch
+    for _ in range(max(warmup, 3)):
+        fn()
+    torch.cuda.synchronize()
+    st = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    e0.record(st)
+    for _ in range(steps):
+        fn()
+    e1.record(st)
+    torch.cuda.synchronize()
+    barrier()
+    return max_over_ranks(e0.elapsed_time(e1), device, world)
 
 
 def _dominant_kernel(kind, s, dev, outs, reps=20):
@@ -610,26 +664,26 @@ def run_coda(a):
                                        "what": "coda_grg_fwd_hg: GEMM1 stores H*g, GEMM2 reads W2 unfolded"}
         del hws
 
-    # The unfused comparison sequence, timed the same way right after.
+    # The unfused comparison sequence, timed the same way right after, and
+    # both paths split into forward and backward (the pages compare each
+    # direction separately).
     unfused = None
-    if kind == "grg" and not a.no_unfused:
-        ustep, ulaunch, uws = _make_unfused_step(s, bwd, dev)
-        for _ in range(max(a.warmup, 3)):
-            ustep()
-        torch.cuda.synchronize()
-        barrier()
-        e0.record(st)
-        for _ in range(a.steps):
-            ustep()
-        e1.record(st)
-        torch.cuda.synchronize()
-        barrier()
-        u_ms = max_over_ranks(e0.elapsed_time(e1), device, world)
+    if kind in ("grg", "swiglu") and not a.no_unfused:
+        ustep, ulaunch, uws = _make_unfused_step(kind, s, bwd, dev)
+        u_ms = _time_loop(ustep, a.steps, a.warmup, device, world, barrier)
         unfused = {"ms_per_step": round(u_ms / a.steps, 4),
                    "value": round(replica_throughput(flops, a.steps, world, u_ms), 2), "unit": "TFLOP/s",
                    "fused_speedup": round(u_ms / ms_max, 4), "gpu_launches_per_step": ulaunch,
                    "what": "same GEMM kernels with plain stores; residual add, RMSNorm, SwiGLU and their backward "
                            "as separate HBM-round-trip kernels"}
+        for dname in ("fwd", "bwd"):
+            ff, uf = getattr(step, dname, None), getattr(ustep, dname, None)
+            if ff is None or uf is None:
+                continue
+            f_ms = _time_loop(ff, a.steps, a.warmup, device, world, barrier)
+            un_ms = _time_loop(uf, a.steps, a.warmup, device, world, barrier)
+            unfused[dname] = {"fused_ms": round(f_ms / a.steps, 4), "unfused_ms": round(un_ms / a.steps, 4),
+                              "speedup": round(un_ms / f_ms, 4)}
         del uws
 
     # Dominant kernel alone (roofline).

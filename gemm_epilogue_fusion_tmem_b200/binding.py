@@ -81,6 +81,9 @@ def library() -> ctypes.CDLL:
             "coda_mlp_block_fwd": (I, [P] * 11 + [I, I, I, I, F, P, S, P]),
             "coda_mlp_block_bwd_workspace_bytes": (S, [I, I, I, I]),
             "coda_mlp_block_bwd": (I, [P] * 16 + [I, I, I, I, P, S, P]),
+            "coda_swiglu_fwd_unfused": (I, [P, P, P, P, P, P, I, I, I, P, S, P]),
+            "coda_swiglu_bwd_unfused_workspace_bytes": (S, [I, I, I]),
+            "coda_swiglu_bwd_unfused": (I, [P, P, P, P, P, P, P, P, P, I, I, I, P, S, P]),
             "coda_grg_fwd_unfused_workspace_bytes": (S, [I, I, I, I]),
             "coda_grg_fwd_unfused": (I, [P] * 10 + [I, I, I, I, F, P, S, P]),
             "coda_grg_bwd_unfused_workspace_bytes": (S, [I, I, I, I]),
@@ -526,4 +529,37 @@ def mlp_block_bwd(dOut, X, W1, H, r, AB, Y, g, W2, Wdown, out: dict | None = Non
                                   _ptr(W2), _ptr(Wdown), _ptr(o["dX"]), _ptr(o["dR"]), _ptr(o["dW1"]), _ptr(o["dW2"]),
                                   _ptr(o["dg"]), _ptr(o["dWdown"]), M, K, d, F, ws.ptr(), ws.nbytes, _stream()),
            "coda_mlp_block_bwd")
+    return o
+
+
+def swiglu_fwd_unfused(X, Wgu, Wdown, out: dict | None = None, ws: Workspace | None = None) -> dict:
+    """The SwiGLU MLP forward operator by operator (measurement only); returns Y, AB, Out."""
+    lib = library()
+    M, d = X.shape
+    F = Wgu.shape[0] // 2
+    _req(X, "X"), _req(Wgu, "Wgu", shape=(2 * F, d)), _req(Wdown, "Wdown", shape=(d, F))
+    o = dict(out or {})
+    for k, shape in (("Y", (M, F)), ("AB", (M, 2 * F)), ("Out", (M, d))):
+        if k not in o:
+            o[k] = torch.empty(*shape, dtype=torch.bfloat16, device=X.device)
+    ws = ws or workspace(lib.coda_gemm_workspace_bytes(), X.device)
+    _check(lib.coda_swiglu_fwd_unfused(_ptr(X), _ptr(Wgu), _ptr(Wdown), _ptr(o["Y"]), _ptr(o["AB"]), _ptr(o["Out"]),
+                                       M, d, F, ws.ptr(), ws.nbytes, _stream()), "coda_swiglu_fwd_unfused")
+    return o
+
+
+def swiglu_bwd_unfused(dOut, X, Wgu, Wdown, Y, AB, out: dict | None = None, ws: Workspace | None = None) -> dict:
+    """The SwiGLU MLP backward operator by operator (measurement only); returns dX, dWgu, dWdown."""
+    lib = library()
+    M, d = X.shape
+    F = Wgu.shape[0] // 2
+    _req(dOut, "dOut", shape=(M, d)), _req(Y, "Y", shape=(M, F)), _req(AB, "AB", shape=(M, 2 * F))
+    o = dict(out or {})
+    for k, shape in (("dX", (M, d)), ("dWgu", (2 * F, d)), ("dWdown", (d, F))):
+        if k not in o:
+            o[k] = torch.empty(*shape, dtype=torch.bfloat16, device=X.device)
+    ws = ws or workspace(lib.coda_swiglu_bwd_unfused_workspace_bytes(M, d, F), X.device)
+    _check(lib.coda_swiglu_bwd_unfused(_ptr(dOut), _ptr(X), _ptr(Wgu), _ptr(Wdown), _ptr(Y), _ptr(AB), _ptr(o["dX"]),
+                                       _ptr(o["dWgu"]), _ptr(o["dWdown"]), M, d, F, ws.ptr(), ws.nbytes, _stream()),
+           "coda_swiglu_bwd_unfused")
     return o

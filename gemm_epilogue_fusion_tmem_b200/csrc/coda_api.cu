@@ -1033,6 +1033,60 @@ coda_status coda_grg_bwd_unfused(const void* dY, const void* dH_in_or_null, cons
 
 }  // extern "C"
 
+// ------------------------------------------------------------------ unfused SwiGLU MLP
+
+extern "C" {
+
+coda_status coda_swiglu_fwd_unfused(const void* X, const void* Wgu, const void* Wdown, void* Y, void* AB, void* Out,
+                                    int M, int d, int F, void* ws, size_t ws_bytes, void* stream) {
+  if (!X || !Wgu || !Wdown || !Y || !AB || !Out || !ws) return CODA_ERR_INVALID_ARG;
+  CODA_TRY(check_swiglu_shapes(M, d, F));
+  const void* ptrs[] = {X, Wgu, Wdown, Y, AB, Out, ws};
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return CODA_ERR_MISALIGNED;
+  if (ws_bytes < coda_gemm_workspace_bytes()) return CODA_ERR_WORKSPACE_TOO_SMALL;
+  int dev;
+  CODA_TRY(current_device(dev));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  CODA_TRY(gemm_store(X, Wgu, AB, M, 2 * F, d, false, false, nullptr, ws, s));
+  const long long ny = (long long)M * F / 8;
+  CODA_TRY(launch_status(launch_ex(unf_swiglu_fwd_kernel, dim3(ew_grid(ny)), dim3(256), 0, s, 1, cbf(AB), bf(Y), F,
+                                   ny)));
+  return gemm_store(Y, Wdown, Out, M, d, F, false, false, nullptr, ws, s);
+}
+
+size_t coda_swiglu_bwd_unfused_workspace_bytes(int M, int d, int F) {
+  (void)d;
+  if (M < 1 || F < 1) return kStatusBytes;
+  return kStatusBytes + align_up((size_t)M * F * 2, 256) + align_up((size_t)M * 2 * F * 2, 256);
+}
+
+coda_status coda_swiglu_bwd_unfused(const void* dOut, const void* X, const void* Wgu, const void* Wdown,
+                                    const void* Y, const void* AB, void* dX, void* dWgu, void* dWdown, int M, int d,
+                                    int F, void* ws, size_t ws_bytes, void* stream) {
+  if (!dOut || !X || !Wgu || !Wdown || !Y || !AB || !dX || !dWgu || !dWdown || !ws) return CODA_ERR_INVALID_ARG;
+  CODA_TRY(check_swiglu_shapes(M, d, F));
+  const void* ptrs[] = {dOut, X, Wgu, Wdown, Y, AB, dX, dWgu, dWdown, ws};
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return CODA_ERR_MISALIGNED;
+  if (ws_bytes < coda_swiglu_bwd_unfused_workspace_bytes(M, d, F)) return CODA_ERR_WORKSPACE_TOO_SMALL;
+  int dev;
+  CODA_TRY(current_device(dev));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* wsb = static_cast<uint8_t*>(ws) + kStatusBytes;
+  __nv_bfloat16* dY = reinterpret_cast<__nv_bfloat16*>(wsb);
+  __nv_bfloat16* dA = reinterpret_cast<__nv_bfloat16*>(wsb + align_up((size_t)M * F * 2, 256));
+  CODA_TRY(gemm_store(dOut, Wdown, dY, M, F, d, false, true, nullptr, ws, s));
+  const long long ny = (long long)M * F / 8;
+  CODA_TRY(launch_status(launch_ex(unf_swiglu_bwd_kernel, dim3(ew_grid(ny)), dim3(256), 0, s, 1,
+                                   (const __nv_bfloat16*)dY, cbf(AB), dA, F, ny)));
+  CODA_TRY(gemm_store(dOut, Y, dWdown, d, F, M, true, true, nullptr, ws, s));
+  CODA_TRY(gemm_store(dA, X, dWgu, 2 * F, d, M, true, true, nullptr, ws, s));
+  return gemm_store(dA, Wgu, dX, M, d, 2 * F, false, true, nullptr, ws, s);
+}
+
+}  // extern "C"
+
 // ------------------------------------------------------------------ forward without allocation
 //
 // For callers that cannot allocate device memory.  The scratch of the GRG

@@ -344,6 +344,19 @@ coda_status coda_grg_bwd_unfused(const void* dY, const void* dH_in_or_null,
                                  int M, int K, int d, int N,
                                  void* ws, size_t ws_bytes, void* stream);
 
+/* The SwiGLU MLP run operator by operator (measurement and error comparison
+ * only): A = X Wgu^T (plain GEMM, stored as AB);  Y = silu(a) * b;
+ * Out = Y Wdown^T;  backward: dY = dOut Wdown (stored);  dA = SwiGLU'(dY, AB);
+ * dWdown = dOut^T Y;  dWgu = dA^T X;  dX = dA Wgu.  Same arguments and shape
+ * rules as coda_swiglu_fwd / coda_swiglu_bwd (AB required). */
+size_t coda_swiglu_bwd_unfused_workspace_bytes(int M, int d, int F);
+coda_status coda_swiglu_fwd_unfused(const void* X, const void* Wgu, const void* Wdown,
+                                    void* Y, void* AB, void* Out,
+                                    int M, int d, int F, void* ws, size_t ws_bytes, void* stream);
+coda_status coda_swiglu_bwd_unfused(const void* dOut, const void* X, const void* Wgu, const void* Wdown,
+                                    const void* Y, const void* AB, void* dX, void* dWgu, void* dWdown,
+                                    int M, int d, int F, void* ws, size_t ws_bytes, void* stream);
+
 /* ---------------------------------------------------------------- forward without any allocation */
 
 /* Upper bound on M * ceil(d / 256) for coda_grg_fwd_prefolded_static: the

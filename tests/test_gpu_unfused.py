@@ -57,3 +57,27 @@ def test_unfused_matches_oracle_and_fused_error_is_comparable(cuda_lib, M, K, d,
         e_f, e_u = _rms_err(fus[k], ref[k]), _rms_err(unf[k], ref[k])
         rms = float(np.sqrt(np.mean(ref[k] ** 2)))
         assert e_f <= 1.5 * e_u + 1e-4 * rms, f"{tag} {k}: fused rms error {e_f:.3g} vs unfused {e_u:.3g}"
+
+
+@pytest.mark.parametrize("M,d,F", [(200, 256, 320), (512, 512, 1024)])
+def test_swiglu_unfused_matches_oracle_and_fused_error_is_comparable(cuda_lib, M, d, F):
+    t = synth.swiglu_inputs(M, d, F, seed=22)
+    td = {k: v.cuda() for k, v in t.items()}
+    fo = cuda_lib.swiglu_fwd(td["X"], td["Wgu"], td["Wdown"])
+    fb = cuda_lib.swiglu_bwd(td["dOut"], td["X"], td["Wgu"], td["Wdown"], fo["Y"], fo["AB"])
+    uo = cuda_lib.swiglu_fwd_unfused(td["X"], td["Wgu"], td["Wdown"])
+    ub = cuda_lib.swiglu_bwd_unfused(td["dOut"], td["X"], td["Wgu"], td["Wdown"], uo["Y"], uo["AB"])
+    torch.cuda.synchronize()
+    X, Wgu, Wdown, dOut = (f64(t[k]) for k in ("X", "Wgu", "Wdown", "dOut"))
+    fwd = O.swiglu_forward(X, Wgu, Wdown)
+    bwd = O.swiglu_backward(dOut, X, Wgu, Wdown, fwd=fwd)
+    ref = {"Y": fwd["Y"], "Out": fwd["Out"], "dX": bwd["dX"], "dWgu": bwd["dWgu"], "dWdown": bwd["dWdown"]}
+    unf = {"Y": uo["Y"], "Out": uo["Out"], **ub}
+    fus = {"Y": fo["Y"], "Out": fo["Out"], **fb}
+    tag = f"swiglu M={M} d={d} F={F}"
+    for k, v in unf.items():
+        assert_pure(v, ref[k], f"unfused {tag} {k}")
+    for k in ref:
+        e_f, e_u = _rms_err(fus[k], ref[k]), _rms_err(unf[k], ref[k])
+        rms = float(np.sqrt(np.mean(ref[k] ** 2)))
+        assert e_f <= 1.5 * e_u + 1e-4 * rms, f"{tag} {k}: fused rms error {e_f:.3g} vs unfused {e_u:.3g}"
