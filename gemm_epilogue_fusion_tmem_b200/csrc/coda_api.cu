@@ -73,9 +73,11 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Row-major bf16 matrix [rows][cols] (cols contiguous), 128-byte swizzled
-// boxes of box_cols x box_rows; out-of-range elements load as zero.
-bool make_tmap(CUtensorMap* m, const void* base, long long rows, long long cols, int box_cols, int box_rows) {
+// Row-major bf16 matrix [rows][cols] (cols contiguous), swizzled boxes of
+// box_cols x box_rows (128-byte swizzle unless given); out-of-range elements
+// load as zero and are not written by stores.
+bool make_tmap(CUtensorMap* m, const void* base, long long rows, long long cols, int box_cols, int box_rows,
+               CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return false;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
@@ -83,7 +85,7 @@ bool make_tmap(CUtensorMap* m, const void* base, long long rows, long long cols,
   cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -211,13 +213,23 @@ coda_status launch_gemm_mode(const CUtensorMap& ta, const CUtensorMap& tb, GemmP
     di.max_clusters[slot] = clusters;
     di.configured[slot] = true;
   }
+  // Output maps for the epilogue's tile stores: 32 x 32 boxes, 64-byte swizzle
+  // (the staging layout).  The second output (a/b or Hg) shares the rows.
+  CUtensorMap to1, to2;
+  std::memset(&to1, 0, sizeof(to1));
+  std::memset(&to2, 0, sizeof(to2));
+  if (p.out != nullptr && !make_tmap(&to1, p.out, p.M, p.ldo, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+    return CODA_ERR_CUDA;
+  const int ld2 = (EPI == EPI_SWIGLU) ? p.ldo2 : p.ldo;
+  if (p.out2 != nullptr && !make_tmap(&to2, p.out2, p.M, ld2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+    return CODA_ERR_CUDA;
   p.kernel_id = (uint32_t)(slot + 1);
   p.wait_limit_ns = g_wait_limit_ns.load();
   if (p.group_m == 0) p.group_m = 1;
   const int tiles = p.num_m_tiles * p.num_n_tiles;
   const int units = std::min(tiles, di.max_clusters[slot]);  // persistent: one tile stream per CTA (pair)
   if (units <= 0) return CODA_OK;
-  if (launch_ex(kern, dim3(units * C::CTAS), dim3(NUM_THREADS), C::SMEM_BYTES, s, C::CTAS, ta, tb, p) !=
+  if (launch_ex(kern, dim3(units * C::CTAS), dim3(NUM_THREADS), C::SMEM_BYTES, s, C::CTAS, ta, tb, to1, to2, p) !=
       cudaSuccess)
     return CODA_ERR_CUDA;
   return cudaPeekAtLastError() == cudaSuccess ? CODA_OK : CODA_ERR_CUDA;

@@ -115,10 +115,65 @@ __device__ __forceinline__ void load32_bf16(const __nv_bfloat16* p, bool valid, 
   }
 }
 
-__device__ __forceinline__ void store32_bf16(__nv_bfloat16* p, const float (&f)[32]) {
+// Per-warp tile store through shared memory: the warp's 32 rows x 32 columns
+// of one output go to a 2 KiB staging tile (64-byte rows, 16-byte chunks
+// swizzled by (row >> 1) & 3, which makes the row-per-thread writes
+// bank-conflict free and matches the tensor map's 64-byte swizzle); one lane
+// then issues a TMA bulk tensor store.  TMA clips rows and columns outside
+// the tensor, so ragged row tiles need no masking.  Up to kEpiTiles tiles per
+// 32-column step; the staging is reused once the previous step's stores have
+// been read.
+constexpr int kEpiTiles = 3;
+constexpr int kEpiTileBytes = 32 * 32 * 2;
+constexpr int kEpiWarpBytes = kEpiTiles * kEpiTileBytes;
+
+struct EpiStore {
+  uint8_t* stg;   // this warp's staging (kEpiWarpBytes, 1024-byte aligned)
+  int lane;
+  int row0;       // first output row of this warp
+  int rows;       // output rows (M); a warp wholly past them stores nothing
+  int n;          // tiles staged in the current step
+  const CUtensorMap* map[kEpiTiles];
+  int col[kEpiTiles];
+
+  __device__ __forceinline__ void begin() {
+    if (lane == 0) bulk_wait_read_all();
+    __syncwarp();
+    n = 0;
+  }
+  __device__ __forceinline__ void put_packed(const uint4 (&q)[4], const CUtensorMap* m, int c) {
+    uint8_t* t = stg + n * kEpiTileBytes + lane * 64;
+    const int sw = (lane >> 1) & 3;
 #pragma unroll
-  for (int j = 0; j < 4; ++j) stg_v4(p + 8 * j, pack8(f + 8 * j));
-}
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t a = smem_u32(t + ((j ^ sw) << 4));
+      asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(q[j].x), "r"(q[j].y), "r"(q[j].z),
+                   "r"(q[j].w)
+                   : "memory");
+    }
+    map[n] = m;
+    col[n] = c;
+    ++n;
+  }
+  __device__ __forceinline__ void put(const float (&f)[32], const CUtensorMap* m, int c) {
+    uint4 q[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) q[j] = pack8(f + 8 * j);
+    put_packed(q, m, c);
+  }
+  __device__ __forceinline__ void flush() {
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0 && row0 < rows) {
+      for (int t = 0; t < n; ++t) tma_store_2d(map[t], stg + t * kEpiTileBytes, col[t], row0);
+      bulk_commit_group();
+    }
+  }
+  __device__ __forceinline__ void finish() {
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
+  }
+};
 
 // Sum of a 32 x 32 block held one row per lane, reduced over the lanes:
 // afterwards v[0] of lane l holds the sum over all lanes of column l.
@@ -141,7 +196,8 @@ __device__ __forceinline__ void warp_column_sums(float (&v)[32], int lane) {
 // (valid when rv), `group32` = (row - lane) / 32 indexes the per-warp partials.
 template <int EPI>
 __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbase, int row, bool rv, int group32,
-                                              int n_blk, int lane) {
+                                              int n_blk, int lane, EpiStore& es, const CUtensorMap* mo1,
+                                              const CUtensorMap* mo2) {
   if constexpr (EPI == EPI_STORE) {
     const int n0 = n_blk * BN;
 #pragma unroll 1
@@ -155,7 +211,9 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbas
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] *= g[i];
       }
-      if (rv) store32_bf16(p.out + (size_t)row * p.ldo + n0 + c, v);
+      es.begin();
+      es.put(v, mo1, n0 + c);
+      es.flush();
     }
   } else if constexpr (EPI == EPI_RESID_RMS) {
     const int n0 = n_blk * BN;
@@ -179,19 +237,17 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbas
 #pragma unroll
         for (int i = 0; i < 8; ++i) ss = fmaf(hb[i], hb[i], ss);
       }
-      if (rv) {
-        __nv_bfloat16* dst = p.out + (size_t)row * p.ldo + n0 + c;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) stg_v4(dst + 8 * j, hq[j]);
-      }
+      es.begin();
+      es.put_packed(hq, mo1, n0 + c);
       if (p.out2 != nullptr) {
         // Activation-side gain: Hg = bf16(H * g), the second GEMM's operand.
         float g[32];
         load32_bf16(p.colvec + n0 + c, true, g);
 #pragma unroll
         for (int i = 0; i < 32; ++i) g[i] *= v[i] + rres[i];
-        if (rv) store32_bf16(p.out2 + (size_t)row * p.ldo + n0 + c, g);
+        es.put(g, mo2, n0 + c);
       }
+      es.flush();
     }
     if (rv && p.part != nullptr) p.part[(size_t)row * p.ld_part + n_blk] = ss;
   } else if constexpr (EPI == EPI_SWIGLU) {
@@ -211,13 +267,13 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbas
         b[i] *= rr;
         y[i] = a[i] * sigmoid_f(a[i]) * b[i];
       }
-      if (rv) {
-        store32_bf16(p.out + (size_t)row * p.ldo + n0 + c, y);
-        if (p.out2 != nullptr) {
-          store32_bf16(p.out2 + (size_t)row * p.ldo2 + n0 + c, a);
-          store32_bf16(p.out2 + (size_t)row * p.ldo2 + p.split + n0 + c, b);
-        }
+      es.begin();
+      es.put(y, mo1, n0 + c);
+      if (p.out2 != nullptr) {
+        es.put(a, mo2, n0 + c);
+        es.put(b, mo2, p.split + n0 + c);
       }
+      es.flush();
     }
   } else if constexpr (EPI == EPI_DN) {
     const int n0 = n_blk * BN;
@@ -240,7 +296,9 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbas
 #pragma unroll
         for (int i = 0; i < 32; ++i) o[i] += e[i];
       }
-      if (rv) store32_bf16(p.out + (size_t)row * p.ldo + n0 + c, o);
+      es.begin();
+      es.put(o, mo1, n0 + c);
+      es.flush();
       // dg partial: sum over this warp's 32 rows of acc * H, per column.
 #pragma unroll
       for (int i = 0; i < 32; ++i) v[i] *= h[i];
@@ -292,7 +350,9 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbas
         if (i == off) g -= 1.f;
         v[i] = g * dl;
       }
-      if (rv) store32_bf16(p.out + (size_t)row * p.ldo + n0 + c, v);
+      es.begin();
+      es.put(v, mo1, n0 + c);
+      es.flush();
     }
   } else if constexpr (EPI == EPI_ROPE) {
     const int n0 = n_blk * BN;
@@ -319,10 +379,10 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbas
             x2[i] = y2;
           }
         }
-        if (rv) {
-          store32_bf16(p.out + (size_t)row * p.ldo + col0 + c, x1);
-          store32_bf16(p.out + (size_t)row * p.ldo + col0 + half + c, x2);
-        }
+        es.begin();
+        es.put(x1, mo1, col0 + c);
+        es.put(x2, mo1, col0 + half + c);
+        es.flush();
       }
     }
   } else if constexpr (EPI == EPI_SWIGLU_BWD) {
@@ -351,11 +411,10 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbas
         a[i] = da * rr;
         b[i] = db * rr;
       }
-      if (rv) {
-        __nv_bfloat16* dst = p.out + (size_t)row * p.ldo + n0 + c;
-        store32_bf16(dst, a);
-        store32_bf16(dst + p.split, b);
-      }
+      es.begin();
+      es.put(a, mo1, n0 + c);
+      es.put(b, mo1, p.split + n0 + c);
+      es.flush();
     }
     if (rv && p.part != nullptr) p.part[(size_t)row * p.ld_part + n_blk] = cpart;
   }
@@ -372,7 +431,8 @@ struct TileCfg {
   static constexpr int A_BYTES = 128 * BK * 2;         // 16 KiB
   static constexpr int B_BYTES = B_ROWS * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+  static constexpr int EPI_BYTES = 4 * kEpiWarpBytes;   // staging for the 4 epilogue warps
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 1024 + 256;
   static constexpr int MMA_M = PAIR ? 256 : 128;
   static constexpr int CTAS = PAIR ? 2 : 1;
 };
@@ -380,6 +440,7 @@ struct TileCfg {
 template <int EPI, bool A_MN, bool B_MN, bool PAIR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmO1, const __grid_constant__ CUtensorMap tmO2,
                    const GemmParams p) {
   using C = TileCfg<PAIR>;
   constexpr int S = C::STAGES;
@@ -387,7 +448,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + S * C::A_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + S * C::B_BYTES);
+  uint8_t* sEpi = sB + S * C::B_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sEpi + C::EPI_BYTES);
   uint64_t* empty = full + S;
   uint64_t* tfull = empty + S;
   uint64_t* tempty = tfull + 2;
@@ -572,6 +634,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else {
     // ---------------------------------------------------------------- epilogue (every CTA)
     const int q = warp & 3;  // TMEM lane quarter this warp may access
+    EpiStore es;
+    es.stg = sEpi + (warp - 2) * kEpiWarpBytes;
+    es.lane = lane;
+    es.rows = p.M;
+    es.n = 0;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = first_tile; tile < num_tiles; tile += tile_step) {
@@ -583,7 +650,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       const uint32_t tbase = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
       const int row0 = m_blk * C::TILE_M + (int)rank * 128 + q * 32;
-      epilogue_tile<EPI>(p, tbase, row0 + lane, row0 + lane < p.M, row0 / 32, n_blk, lane);
+      es.row0 = row0;
+      epilogue_tile<EPI>(p, tbase, row0 + lane, row0 + lane < p.M, row0 / 32, n_blk, lane, es, &tmO1, &tmO2);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -593,6 +661,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
+    es.finish();  // every tile store has completed before the CTA's shared memory is released
   }
 
   tc_fence_before();
