@@ -23,6 +23,7 @@ _c_int = ctypes.c_int
 _c_size_t = ctypes.c_size_t
 _c_float = ctypes.c_float
 
+CODA_ERR_INVALID_ARG = 1
 CODA_ERR_DEVICE_TIMEOUT = 7
 
 
@@ -56,6 +57,7 @@ def library() -> ctypes.CDLL:
             "coda_status_query": (I, [P, P, ctypes.POINTER(ctypes.c_uint32)]),
             "coda_set_wait_limit_ns": (None, [ctypes.c_uint64]),
             "coda_selftest_wait_timeout": (I, [P, ctypes.c_uint64, P]),
+            "coda_profile_arm": (I, [I, P, P]),
             "coda_gemm_workspace_bytes": (S, []),
             "coda_gemm": (I, [P, P, P, I, I, I, I, I, P, S, P]),
             "coda_fold_gain": (I, [P, P, P, I, I, P]),
@@ -171,6 +173,22 @@ def workspace(nbytes: int, device=None) -> Workspace:
 
 def set_wait_limit_ns(ns: int) -> None:
     library().coda_set_wait_limit_ns(int(ns))
+
+
+EPI_STORE, EPI_RESID_RMS, EPI_SWIGLU, EPI_DN, EPI_SWIGLU_BWD, EPI_XENT, EPI_XENT_BWD, EPI_ROPE = range(8)
+
+
+def profile_arm(epilogue: int, start=None, stop=None) -> None:
+    """Arm a one-shot torch.cuda.Event pair around the next GEMM launch with this
+    epilogue (EPI_*) from this thread; no events disarms."""
+    def handle(ev):
+        if ev is None:
+            return None
+        if ev.cuda_event == 0:  # torch creates the CUDA event at its first record
+            ev.record()
+        return ctypes.c_void_p(ev.cuda_event)
+
+    _check(library().coda_profile_arm(int(epilogue), handle(start), handle(stop)), "coda_profile_arm")
 
 
 def selftest_wait_timeout(ws: Workspace, limit_ns: int) -> None:

@@ -20,6 +20,13 @@ namespace {
 constexpr size_t kStatusBytes = 256;
 std::atomic<unsigned long long> g_wait_limit_ns{4000000000ull};
 
+// One-shot event pair armed by coda_profile_arm, per host thread.
+struct ProfileArm {
+  int epi = -1;
+  cudaEvent_t start = nullptr, stop = nullptr;
+};
+thread_local ProfileArm g_prof;
+
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline int cdiv(long long a, long long b) { return (int)((a + b - 1) / b); }
@@ -229,9 +236,15 @@ coda_status launch_gemm_mode(const CUtensorMap& ta, const CUtensorMap& tb, GemmP
   const int tiles = p.num_m_tiles * p.num_n_tiles;
   const int units = std::min(tiles, di.max_clusters[slot]);  // persistent: one tile stream per CTA (pair)
   if (units <= 0) return CODA_OK;
+  const bool timed = g_prof.epi == EPI;
+  if (timed && cudaEventRecord(g_prof.start, s) != cudaSuccess) return CODA_ERR_CUDA;
   if (launch_ex(kern, dim3(units * C::CTAS), dim3(NUM_THREADS), C::SMEM_BYTES, s, C::CTAS, ta, tb, to1, to2, p) !=
       cudaSuccess)
     return CODA_ERR_CUDA;
+  if (timed) {
+    g_prof.epi = -1;
+    if (cudaEventRecord(g_prof.stop, s) != cudaSuccess) return CODA_ERR_CUDA;
+  }
   return cudaPeekAtLastError() == cudaSuccess ? CODA_OK : CODA_ERR_CUDA;
 }
 
@@ -329,6 +342,23 @@ void coda_set_wait_limit_ns(uint64_t ns) {
   ns = std::max<uint64_t>(ns, 1000ull);
   ns = std::min<uint64_t>(ns, 60000000000ull);
   g_wait_limit_ns.store(ns);
+}
+
+coda_status coda_profile_arm(int epilogue, void* ev_start, void* ev_stop) {
+  static_assert(CODA_EPI_STORE == EPI_STORE && CODA_EPI_RESID_RMS == EPI_RESID_RMS && CODA_EPI_SWIGLU == EPI_SWIGLU &&
+                    CODA_EPI_DN == EPI_DN && CODA_EPI_SWIGLU_BWD == EPI_SWIGLU_BWD && CODA_EPI_XENT == EPI_XENT &&
+                    CODA_EPI_XENT_BWD == EPI_XENT_BWD && CODA_EPI_ROPE == EPI_ROPE,
+                "public epilogue ids");
+  if (ev_start == nullptr && ev_stop == nullptr) {
+    g_prof = ProfileArm();
+    return CODA_OK;
+  }
+  if (ev_start == nullptr || ev_stop == nullptr || epilogue < CODA_EPI_STORE || epilogue > CODA_EPI_ROPE)
+    return CODA_ERR_INVALID_ARG;
+  g_prof.epi = epilogue;
+  g_prof.start = static_cast<cudaEvent_t>(ev_start);
+  g_prof.stop = static_cast<cudaEvent_t>(ev_stop);
+  return CODA_OK;
 }
 
 coda_status coda_selftest_wait_timeout(void* ws, uint64_t limit_ns, void* stream) {

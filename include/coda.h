@@ -90,6 +90,26 @@ void coda_set_wait_limit_ns(uint64_t ns);
  * it with coda_status_clear. */
 coda_status coda_selftest_wait_timeout(void* ws, uint64_t limit_ns, void* stream);
 
+/* Kernel timing hook.  Arms a one-shot pair of CUDA events around the next
+ * launch, from the calling host thread, of a GEMM whose epilogue is
+ * `epilogue` (one of CODA_EPI_*), whichever entry point makes it: ev_start is
+ * recorded on that launch's stream immediately before the kernel and ev_stop
+ * immediately after, then the hook disarms itself.  ev_start and ev_stop are
+ * cudaEvent_t handles created and owned by the caller (timing enabled); the
+ * library only records them.  Both NULL disarms.  Returns CODA_ERR_INVALID_ARG
+ * for an unknown epilogue or a single NULL event.  Recording the events takes
+ * the place of the programmatic (PDL) overlap between that kernel and its
+ * neighbours, so an armed launch can start a few microseconds later. */
+#define CODA_EPI_STORE 0      /* plain store (optional column scale) */
+#define CODA_EPI_RESID_RMS 1  /* + residual, H, partial sums of squares */
+#define CODA_EPI_SWIGLU 2     /* r scaling + SwiGLU (the gate/up GEMM) */
+#define CODA_EPI_DN 3         /* RMSNorm correction + dg partials (backward) */
+#define CODA_EPI_SWIGLU_BWD 4 /* SwiGLU backward (the down GEMM's backward) */
+#define CODA_EPI_XENT 5       /* online max / sum-exp (the logits GEMM) */
+#define CODA_EPI_XENT_BWD 6   /* softmax - one-hot, dlogits */
+#define CODA_EPI_ROPE 7       /* rotary embedding (the QKV GEMM) */
+coda_status coda_profile_arm(int epilogue, void* ev_start, void* ev_stop);
+
 /* ---------------------------------------------------------------- building block */
 
 /* C[M,N] (bf16) = op(A) * op(B)^T with fp32 accumulation on tcgen05 tensor cores.

@@ -47,3 +47,16 @@ def test_status_strings_round_trip():
     assert "timed out" in B._status_string(B.CODA_ERR_DEVICE_TIMEOUT)
     err = B.CodaError(3, "coda_gemm")
     assert err.status == 3 and "16-byte" in str(err)
+
+
+def test_profile_hook_argument_checks():
+    """coda_profile_arm validates its arguments without touching the GPU."""
+    import ctypes
+    lib = B.library()
+    fake = ctypes.c_void_p(1)  # never recorded: every call below is refused or disarms
+    assert lib.coda_profile_arm(99, fake, fake) == B.CODA_ERR_INVALID_ARG
+    assert lib.coda_profile_arm(-1, fake, fake) == B.CODA_ERR_INVALID_ARG
+    assert lib.coda_profile_arm(B.EPI_SWIGLU, fake, None) == B.CODA_ERR_INVALID_ARG
+    assert lib.coda_profile_arm(B.EPI_SWIGLU, None, fake) == B.CODA_ERR_INVALID_ARG
+    assert lib.coda_profile_arm(B.EPI_SWIGLU, None, None) == 0  # disarm
+    assert (B.EPI_STORE, B.EPI_SWIGLU, B.EPI_XENT, B.EPI_ROPE) == (0, 2, 5, 7)

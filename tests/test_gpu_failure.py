@@ -47,3 +47,32 @@ def test_status_is_sticky_until_cleared(cuda_lib):
     assert ws.query()[0] == CODA_ERR_DEVICE_TIMEOUT  # reading does not clear it
     ws.clear()
     assert ws.query() == (0, 0)
+
+
+def test_profile_hook_times_one_launch(cuda_lib):
+    """The timing hook records its event pair around exactly one launch of the
+    armed epilogue and then disarms: a second launch leaves the events alone,
+    and a launch with another epilogue never triggers it."""
+    B = cuda_lib
+    M, F, K = 2048, 4096, 4096
+    A = torch.randn(M, K, device="cuda").to(torch.bfloat16)
+    W = (torch.randn(2 * F, K, device="cuda") * K ** -0.5).to(torch.bfloat16)
+    o = B.gemm_swiglu(A, W)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    B.profile_arm(B.EPI_XENT, ev[0], ev[1])  # another epilogue: not triggered by the SwiGLU GEMM
+    B.gemm_swiglu(A, W, out=o)
+    ev[2].record()
+    torch.cuda.synchronize()
+    assert ev[1].elapsed_time(ev[2]) > 0.01  # both recorded at arming, before the launch
+    B.profile_arm(B.EPI_SWIGLU, ev[0], ev[1])
+    B.gemm_swiglu(A, W, out=o)
+    B.gemm_swiglu(A, W, out=o)  # the hook is one-shot: this launch records nothing
+    ev[2].record()
+    torch.cuda.synchronize()
+    k = ev[0].elapsed_time(ev[1])
+    after = ev[1].elapsed_time(ev[2])
+    flops = 2.0 * M * K * 2 * F
+    assert 0.005 < k < 5.0, k
+    assert flops / (k / 1e3) < 3.0e15  # below any B200 bf16 rate: the pair spans the kernel
+    assert after > 0.5 * k, (k, after)
+    B.profile_arm(B.EPI_SWIGLU)
