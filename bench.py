@@ -471,6 +471,65 @@ def _time_loop(fn, steps, warmup, device, world, barrier):
     return max_over_ranks(e0.elapsed_time(e1), device, world)
 
 
+def _grg_kernels(s, bwd):
+    """The block's kernels in launch order with their algorithmic work per launch:
+    (hook id, name, bound, amount) with FLOPs for tensor-bound GEMMs and
+    compulsory HBM bytes for the light passes."""
+    M, K, d, F = s["M"], s["K"], s["d"], s["F"]
+    N = 2 * F
+    T = -(-d // 256)  # partial sums per row (one per 256-column tile)
+    ks = [(16, "fold_gain (W2g = W2 diag g)", "hbm", 4.0 * N * d + 2.0 * d),
+          (1, "GEMM1 + residual + partial sums", "tensor", 2.0 * M * K * d),
+          (17, "row reduce -> r", "hbm", 4.0 * M * T + 4.0 * M),
+          (2, "GEMM2 + r + SwiGLU", "tensor", 2.0 * M * d * N)]
+    if bwd:
+        rows = -(-M // 256) * 256 // 32  # dg partial rows: one per 32 output rows
+        ks += [(18, "SwiGLU bwd + row coefficient", "hbm", 2.0 * M * F + 4.0 * M * N + 8.0 * M),
+               (3, "dn GEMM + RMSNorm correction + dg partials", "tensor", 2.0 * M * N * d),
+               (19, "column reduce -> dg", "hbm", 4.0 * rows * d + 4.0 * d),
+               (0, "dW2 = g (dA'^T H)", "tensor", 2.0 * N * d * M),
+               (0, "dX = dH W1", "tensor", 2.0 * M * K * d),
+               (0, "dW1 = dH^T X", "tensor", 2.0 * d * K * M)]
+    return ks
+
+
+def _kernel_breakdown(kind, s, bwd, step, reps=10):
+    """Every kernel of the block's step timed through the library's event hook
+    over `reps` extra steps (outside the timed region: the events take the
+    place of the PDL overlap at every boundary), against the measured peaks."""
+    if kind != "grg":
+        return None
+    import torch
+    from gemm_epilogue_fusion_tmem_b200 import binding as B
+    peaks, src = _peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    tc = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    ks = _grg_kernels(s, bwd)
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in ks]
+          for _ in range(reps)]
+    torch.cuda.synchronize()
+    for r in range(reps):
+        for (kid, _, _, _), (x, y) in zip(ks, ev[r]):
+            B.profile_arm(kid, x, y)
+        step()
+    torch.cuda.synchronize()
+    B.profile_arm(0)
+    out = []
+    for i, (kid, name, bound, amount) in enumerate(ks):
+        ms = sum(ev[r][i][0].elapsed_time(ev[r][i][1]) for r in range(reps)) / reps
+        if bound == "tensor":
+            ach = amount / (ms / 1e3) / 1e12
+            out.append({"kernel": name, "ms": round(ms, 4), "bound": "tensor", "TFLOP": round(amount / 1e12, 4),
+                        "achieved_TFLOP/s": round(ach, 1), "frac": round(ach / tc, 4)})
+        else:
+            ach = amount / (ms / 1e3) / 1e9
+            out.append({"kernel": name, "ms": round(ms, 4), "bound": "hbm", "MB": round(amount / 1e6, 2),
+                        "achieved_GB/s": round(ach, 1), "frac": round(ach / hbm, 4)})
+    return {"steps": reps, "peaks": f"{src}: sustained bf16 {tc} TFLOP/s, HBM copy {hbm} GB/s",
+            "note": "each kernel inside its own CUDA-event pair (no PDL overlap at its boundaries)",
+            "kernels": out, "sum_ms": round(sum(k["ms"] for k in out), 4)}
+
+
 # Epilogue of the dominant GEMM per workload kind (the launch the timing hook arms).
 DOMINANT_EPI = {"grg": 2, "swiglu": 2, "block": 2, "xent": 5, "rope": 7}
 
@@ -705,6 +764,9 @@ def run_coda(a):
                           "frac": round(alone / burst, 4),
                           "peak_source": f"{peaks_src} burst bf16 (kernel timed alone, after warm-up)"}}
 
+    # Every kernel of the step timed on its own (light passes in GB/s against HBM).
+    breakdown = _kernel_breakdown(kind, s, bwd, step)
+
     # End to end through the public API with host buffers: every step copies its
     # inputs from pinned host memory and its results back, inside the timed
     # region.  Inputs and outputs are double-buffered and the copies run on their
@@ -737,6 +799,7 @@ def run_coda(a):
                        "l2": "inputs larger than L2 (step working set > 1 GB), no flush",
                        "flops_per_step": flops, "frac_of_sustained_bf16_peak": round(frac_step, 4)},
             "roofline": roofline,
+            "kernels": breakdown,
             "cpu_baseline": cpu,
             "unfused": unfused,
             "variants": variants or None,

@@ -175,12 +175,16 @@ def set_wait_limit_ns(ns: int) -> None:
     library().coda_set_wait_limit_ns(int(ns))
 
 
+# Kernel ids of the timing hook (coda_profile_arm): GEMMs by epilogue, light passes from 16.
 EPI_STORE, EPI_RESID_RMS, EPI_SWIGLU, EPI_DN, EPI_SWIGLU_BWD, EPI_XENT, EPI_XENT_BWD, EPI_ROPE = range(8)
+(KERNEL_FOLD_GAIN, KERNEL_RMS_ROWREDUCE, KERNEL_SWIGLU_BWD_ROWSTAT, KERNEL_COL_REDUCE, KERNEL_ROWCOEF_REDUCE,
+ KERNEL_XENT_REDUCE, KERNEL_ROPE_UNROTATE) = range(16, 23)
 
 
-def profile_arm(epilogue: int, start=None, stop=None) -> None:
-    """Arm a one-shot torch.cuda.Event pair around the next GEMM launch with this
-    epilogue (EPI_*) from this thread; no events disarms."""
+def profile_arm(kernel: int, start=None, stop=None) -> None:
+    """Arm a one-shot torch.cuda.Event pair around the next launch, from this
+    thread, of the kernel `kernel` names (EPI_* or KERNEL_*); pairs armed for
+    the same kernel fire on its successive launches.  No events disarms all."""
     def handle(ev):
         if ev is None:
             return None
@@ -188,7 +192,7 @@ def profile_arm(epilogue: int, start=None, stop=None) -> None:
             ev.record()
         return ctypes.c_void_p(ev.cuda_event)
 
-    _check(library().coda_profile_arm(int(epilogue), handle(start), handle(stop)), "coda_profile_arm")
+    _check(library().coda_profile_arm(int(kernel), handle(start), handle(stop)), "coda_profile_arm")
 
 
 def selftest_wait_timeout(ws: Workspace, limit_ns: int) -> None:

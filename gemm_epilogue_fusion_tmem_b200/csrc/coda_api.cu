@@ -8,6 +8,7 @@
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
+#include <initializer_list>
 
 #include "coda.h"
 #include "coda_aux.cuh"
@@ -20,12 +21,28 @@ namespace {
 constexpr size_t kStatusBytes = 256;
 std::atomic<unsigned long long> g_wait_limit_ns{4000000000ull};
 
-// One-shot event pair armed by coda_profile_arm, per host thread.
-struct ProfileArm {
-  int epi = -1;
-  cudaEvent_t start = nullptr, stop = nullptr;
+// One-shot event pairs armed by coda_profile_arm, per host thread, in arming order.
+struct ProfileSlot {
+  int kernel;
+  cudaEvent_t start, stop;
 };
-thread_local ProfileArm g_prof;
+constexpr int kProfileSlots = 16;
+thread_local ProfileSlot g_prof[kProfileSlots];
+thread_local int g_prof_n = 0;
+thread_local int g_launch_tag = -1;  // the GEMM launcher's epilogue id around its launch
+
+// Remove and return the first pair armed for kernel id `tag`.
+bool profile_take(int tag, cudaEvent_t& start, cudaEvent_t& stop) {
+  for (int i = 0; i < g_prof_n; ++i) {
+    if (g_prof[i].kernel != tag) continue;
+    start = g_prof[i].start;
+    stop = g_prof[i].stop;
+    for (int j = i + 1; j < g_prof_n; ++j) g_prof[j - 1] = g_prof[j];
+    --g_prof_n;
+    return true;
+  }
+  return false;
+}
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -128,7 +145,22 @@ bool use_pdl() {
   return v;
 }
 
-// Launch with the optional cluster size and the PDL attribute.
+// Timing-hook id of a light-pass kernel (-1 for kernels the hook does not name).
+template <typename Fn>
+int aux_tag(Fn kern) {
+  const void* f = reinterpret_cast<const void*>(kern);
+  if (f == reinterpret_cast<const void*>(fold_gain_kernel)) return CODA_KERNEL_FOLD_GAIN;
+  if (f == reinterpret_cast<const void*>(rms_rowreduce_kernel)) return CODA_KERNEL_RMS_ROWREDUCE;
+  if (f == reinterpret_cast<const void*>(swiglu_bwd_rowstat_kernel)) return CODA_KERNEL_SWIGLU_BWD_ROWSTAT;
+  if (f == reinterpret_cast<const void*>(col_reduce_kernel)) return CODA_KERNEL_COL_REDUCE;
+  if (f == reinterpret_cast<const void*>(rowcoef_reduce_kernel)) return CODA_KERNEL_ROWCOEF_REDUCE;
+  if (f == reinterpret_cast<const void*>(xent_reduce_kernel)) return CODA_KERNEL_XENT_REDUCE;
+  if (f == reinterpret_cast<const void*>(rope_unrotate_kernel)) return CODA_KERNEL_ROPE_UNROTATE;
+  return -1;
+}
+
+// Launch with the optional cluster size and the PDL attribute, inside the
+// timing hook's event pair when one is armed for this kernel.
 template <typename... KArgs, typename... Args>
 cudaError_t launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, int cluster,
                       Args&&... args) {
@@ -154,7 +186,15 @@ cudaError_t launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = n;
-  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+  cudaEvent_t ev0 = nullptr, ev1 = nullptr;
+  const bool timed = g_prof_n > 0 && profile_take(g_launch_tag >= 0 ? g_launch_tag : aux_tag(kern), ev0, ev1);
+  if (timed) {
+    const cudaError_t e = cudaEventRecord(ev0, s);
+    if (e != cudaSuccess) return e;
+  }
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+  if (timed && e == cudaSuccess) e = cudaEventRecord(ev1, s);
+  return e;
 }
 
 // Rasterisation.  Concurrent tiles read the same k-slices at about the same
@@ -236,15 +276,11 @@ coda_status launch_gemm_mode(const CUtensorMap& ta, const CUtensorMap& tb, GemmP
   const int tiles = p.num_m_tiles * p.num_n_tiles;
   const int units = std::min(tiles, di.max_clusters[slot]);  // persistent: one tile stream per CTA (pair)
   if (units <= 0) return CODA_OK;
-  const bool timed = g_prof.epi == EPI;
-  if (timed && cudaEventRecord(g_prof.start, s) != cudaSuccess) return CODA_ERR_CUDA;
-  if (launch_ex(kern, dim3(units * C::CTAS), dim3(NUM_THREADS), C::SMEM_BYTES, s, C::CTAS, ta, tb, to1, to2, p) !=
-      cudaSuccess)
-    return CODA_ERR_CUDA;
-  if (timed) {
-    g_prof.epi = -1;
-    if (cudaEventRecord(g_prof.stop, s) != cudaSuccess) return CODA_ERR_CUDA;
-  }
+  g_launch_tag = EPI;
+  const cudaError_t e =
+      launch_ex(kern, dim3(units * C::CTAS), dim3(NUM_THREADS), C::SMEM_BYTES, s, C::CTAS, ta, tb, to1, to2, p);
+  g_launch_tag = -1;
+  if (e != cudaSuccess) return CODA_ERR_CUDA;
   return cudaPeekAtLastError() == cudaSuccess ? CODA_OK : CODA_ERR_CUDA;
 }
 
@@ -344,20 +380,19 @@ void coda_set_wait_limit_ns(uint64_t ns) {
   g_wait_limit_ns.store(ns);
 }
 
-coda_status coda_profile_arm(int epilogue, void* ev_start, void* ev_stop) {
+coda_status coda_profile_arm(int kernel, void* ev_start, void* ev_stop) {
   static_assert(CODA_EPI_STORE == EPI_STORE && CODA_EPI_RESID_RMS == EPI_RESID_RMS && CODA_EPI_SWIGLU == EPI_SWIGLU &&
                     CODA_EPI_DN == EPI_DN && CODA_EPI_SWIGLU_BWD == EPI_SWIGLU_BWD && CODA_EPI_XENT == EPI_XENT &&
                     CODA_EPI_XENT_BWD == EPI_XENT_BWD && CODA_EPI_ROPE == EPI_ROPE,
                 "public epilogue ids");
   if (ev_start == nullptr && ev_stop == nullptr) {
-    g_prof = ProfileArm();
+    g_prof_n = 0;
     return CODA_OK;
   }
-  if (ev_start == nullptr || ev_stop == nullptr || epilogue < CODA_EPI_STORE || epilogue > CODA_EPI_ROPE)
-    return CODA_ERR_INVALID_ARG;
-  g_prof.epi = epilogue;
-  g_prof.start = static_cast<cudaEvent_t>(ev_start);
-  g_prof.stop = static_cast<cudaEvent_t>(ev_stop);
+  const bool known = (kernel >= CODA_EPI_STORE && kernel <= CODA_EPI_ROPE) ||
+                     (kernel >= CODA_KERNEL_FOLD_GAIN && kernel <= CODA_KERNEL_ROPE_UNROTATE);
+  if (ev_start == nullptr || ev_stop == nullptr || !known || g_prof_n >= kProfileSlots) return CODA_ERR_INVALID_ARG;
+  g_prof[g_prof_n++] = ProfileSlot{kernel, static_cast<cudaEvent_t>(ev_start), static_cast<cudaEvent_t>(ev_stop)};
   return CODA_OK;
 }
 
@@ -388,10 +423,36 @@ coda_status coda_status_query(const void* ws, void* stream, uint32_t* detail) {
 
 // ------------------------------------------------------------------ plain GEMM
 
+namespace coda {
+namespace {
+// An empty batch (M == 0) has no row to read or write; each weight gradient
+// is then a sum over no rows and is written as zeros.  Row-sized pointers may
+// be NULL; the weight-gradient pointers must be valid.
+struct ZeroSpan {
+  void* p;
+  size_t bytes;
+};
+coda_status zero_fill(std::initializer_list<ZeroSpan> spans, void* stream) {
+  for (const ZeroSpan& z : spans) {
+    if (z.p == nullptr) return CODA_ERR_INVALID_ARG;
+    if (!aligned16(z.p)) return CODA_ERR_MISALIGNED;
+  }
+  int dev;
+  CODA_TRY(current_device(dev));
+  for (const ZeroSpan& z : spans)
+    if (cudaMemsetAsync(z.p, 0, z.bytes, static_cast<cudaStream_t>(stream)) != cudaSuccess) return CODA_ERR_CUDA;
+  return CODA_OK;
+}
+}  // namespace
+}  // namespace coda
+
 size_t coda_gemm_workspace_bytes(void) { return kStatusBytes; }
 
 coda_status coda_gemm(const void* A, const void* B, void* C, int M, int N, int K, int a_mn_major, int b_mn_major,
                       void* ws, size_t ws_bytes, void* stream) {
+  if (M < 0 || N < 0 || K < 0) return CODA_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return CODA_OK;                               // empty output
+  if (K == 0) return zero_fill({{C, (size_t)M * N * 2}}, stream);     // empty sums
   if (!A || !B || !C || !ws) return CODA_ERR_INVALID_ARG;
   if (M < 1 || N < 1 || K < 1) return CODA_ERR_INVALID_ARG;
   if (N % 32 != 0) return CODA_ERR_UNSUPPORTED_SHAPE;
@@ -406,6 +467,8 @@ coda_status coda_gemm(const void* A, const void* B, void* C, int M, int N, int K
 
 coda_status coda_gemm_swiglu(const void* A, const void* Wgu, const float* r_or_null, void* Y, void* AB_or_null,
                              int M, int K, int F, void* ws, size_t ws_bytes, void* stream) {
+  if (M == 0) return (K < 1 || F < 1) ? CODA_ERR_INVALID_ARG
+                    : (K % 64 != 0 || F % 64 != 0) ? CODA_ERR_UNSUPPORTED_SHAPE : CODA_OK;
   if (!A || !Wgu || !Y || !ws) return CODA_ERR_INVALID_ARG;
   if (M < 1 || K < 1 || F < 1) return CODA_ERR_INVALID_ARG;
   if (K % 64 != 0 || F % 64 != 0) return CODA_ERR_UNSUPPORTED_SHAPE;
@@ -465,6 +528,7 @@ size_t coda_grg_fwd_workspace_bytes(int M, int K, int d, int N, int prefolded) {
 coda_status coda_grg_fwd(const void* X, const void* W1, const void* R, const void* g, const void* W2,
                          const void* W2g_or_null, void* H, float* r, void* Y, void* AB_or_null, int M, int K, int d,
                          int N, float eps, void* ws, size_t ws_bytes, void* stream) {
+  if (M == 0) return !(eps > 0.f) ? CODA_ERR_INVALID_ARG : check_grg_shapes(1, K, d, N);  // empty batch
   if (!X || !W1 || !R || !H || !r || !Y || !ws) return CODA_ERR_INVALID_ARG;
   if (W2g_or_null == nullptr && (!g || !W2)) return CODA_ERR_INVALID_ARG;
   if (!(eps > 0.f)) return CODA_ERR_INVALID_ARG;
@@ -526,6 +590,7 @@ size_t coda_grg_fwd_hg_workspace_bytes(int M, int K, int d, int N, int hg_given)
 coda_status coda_grg_fwd_hg(const void* X, const void* W1, const void* R, const void* g, const void* W2, void* H,
                             void* Hg_or_null, float* r, void* Y, void* AB_or_null, int M, int K, int d, int N,
                             float eps, void* ws, size_t ws_bytes, void* stream) {
+  if (M == 0) return !(eps > 0.f) ? CODA_ERR_INVALID_ARG : check_grg_shapes(1, K, d, N);  // empty batch
   if (!X || !W1 || !R || !g || !W2 || !H || !r || !Y || !ws) return CODA_ERR_INVALID_ARG;
   if (!(eps > 0.f)) return CODA_ERR_INVALID_ARG;
   CODA_TRY(check_grg_shapes(M, K, d, N));
@@ -625,6 +690,10 @@ coda_status coda_grg_bwd(const void* dY, const void* dH_in_or_null, const void* 
                          const float* r, const void* AB, const void* g, const void* W2, void* dX, void* dR,
                          void* dW1, void* dW2, float* dg, int M, int K, int d, int N, void* ws, size_t ws_bytes,
                          void* stream) {
+  if (M == 0) {  // empty batch: zero weight gradients
+    CODA_TRY(check_grg_shapes(1, K, d, N));
+    return zero_fill({{dW1, (size_t)d * K * 2}, {dW2, (size_t)N * d * 2}, {dg, (size_t)d * 4}}, stream);
+  }
   if (!dY || !X || !W1 || !H || !r || !AB || !g || !W2 || !dX || !dR || !dW1 || !dW2 || !dg || !ws)
     return CODA_ERR_INVALID_ARG;
   CODA_TRY(check_grg_shapes(M, K, d, N));
@@ -666,6 +735,7 @@ size_t coda_swiglu_fwd_workspace_bytes(int M, int d, int F) {
 
 coda_status coda_swiglu_fwd(const void* X, const void* Wgu, const void* Wdown, void* Y, void* AB_or_null,
                             void* Out, int M, int d, int F, void* ws, size_t ws_bytes, void* stream) {
+  if (M == 0) return check_swiglu_shapes(1, d, F);  // empty batch
   if (!X || !Wgu || !Wdown || !Y || !Out || !ws) return CODA_ERR_INVALID_ARG;
   CODA_TRY(check_swiglu_shapes(M, d, F));
   const void* ptrs[] = {X, Wgu, Wdown, Y, AB_or_null, Out, ws};
@@ -688,6 +758,10 @@ size_t coda_swiglu_bwd_workspace_bytes(int M, int d, int F) {
 coda_status coda_swiglu_bwd(const void* dOut, const void* X, const void* Wgu, const void* Wdown, const void* Y,
                             const void* AB, void* dX, void* dWgu, void* dWdown, int M, int d, int F, void* ws,
                             size_t ws_bytes, void* stream) {
+  if (M == 0) {  // empty batch: zero weight gradients
+    CODA_TRY(check_swiglu_shapes(1, d, F));
+    return zero_fill({{dWgu, (size_t)2 * F * d * 2}, {dWdown, (size_t)d * F * 2}}, stream);
+  }
   if (!dOut || !X || !Wgu || !Wdown || !Y || !AB || !dX || !dWgu || !dWdown || !ws) return CODA_ERR_INVALID_ARG;
   CODA_TRY(check_swiglu_shapes(M, d, F));
   const void* ptrs[] = {dOut, X, Wgu, Wdown, Y, AB, dX, dWgu, dWdown, ws};
@@ -733,8 +807,8 @@ size_t coda_xent_fwd_workspace_bytes(int M, int d, int V) {
 
 namespace {
 coda_status check_xent(const void* X, const void* W, const void* t, int M, int d, int V) {
-  if (!X || !W || !t) return CODA_ERR_INVALID_ARG;
-  if (M < 1 || d < 1 || V < 1) return CODA_ERR_INVALID_ARG;
+  if (!W || (M > 0 && (!X || !t))) return CODA_ERR_INVALID_ARG;
+  if (M < 0 || d < 1 || V < 1) return CODA_ERR_INVALID_ARG;
   if (d % 64 != 0 || V % 64 != 0) return CODA_ERR_UNSUPPORTED_SHAPE;
   return CODA_OK;
 }
@@ -743,6 +817,7 @@ coda_status check_xent(const void* X, const void* W, const void* t, int M, int d
 coda_status coda_xent_fwd(const void* X, const void* W, const int32_t* targets, float* loss, float* lse, int M,
                           int d, int V, void* ws, size_t ws_bytes, void* stream) {
   CODA_TRY(check_xent(X, W, targets, M, d, V));
+  if (M == 0) return CODA_OK;  // empty batch
   if (!loss || !lse || !ws) return CODA_ERR_INVALID_ARG;
   const void* ptrs[] = {X, W, targets, loss, lse, ws};
   for (const void* q : ptrs)
@@ -784,6 +859,7 @@ coda_status coda_xent_bwd(const void* X, const void* W, const int32_t* targets, 
                           const float* dloss, void* dX, void* dW, int M, int d, int V, void* ws, size_t ws_bytes,
                           void* stream) {
   CODA_TRY(check_xent(X, W, targets, M, d, V));
+  if (M == 0) return zero_fill({{dW, (size_t)V * d * 2}}, stream);  // empty batch: zero weight gradient
   if (!lse || !dloss || !dX || !dW || !ws) return CODA_ERR_INVALID_ARG;
   const void* ptrs[] = {X, W, targets, lse, dloss, dX, dW, ws};
   for (const void* q : ptrs)
@@ -824,6 +900,7 @@ size_t coda_mlp_block_fwd_workspace_bytes(int M, int K, int d, int F) {
 coda_status coda_mlp_block_fwd(const void* X, const void* W1, const void* R, const void* g, const void* W2,
                                const void* Wdown, void* H, float* r, void* Y, void* AB, void* Out, int M, int K,
                                int d, int F, float eps, void* ws, size_t ws_bytes, void* stream) {
+  if (M == 0) return !(eps > 0.f) ? CODA_ERR_INVALID_ARG : check_grg_shapes(1, K, d, 2 * F);  // empty batch
   if (!Wdown || !Out || !AB) return CODA_ERR_INVALID_ARG;
   if (!aligned16(Wdown) || !aligned16(Out)) return CODA_ERR_MISALIGNED;
   // Validates every other argument and runs the block's forward.
@@ -869,6 +946,12 @@ coda_status coda_mlp_block_bwd(const void* dOut, const void* X, const void* W1, 
                                const void* AB, const void* Y, const void* g, const void* W2, const void* Wdown,
                                void* dX, void* dR, void* dW1, void* dW2, float* dg, void* dWdown, int M, int K, int d,
                                int F, void* ws, size_t ws_bytes, void* stream) {
+  if (M == 0) {  // empty batch: zero weight gradients
+    CODA_TRY(check_grg_shapes(1, K, d, 2 * F));
+    return zero_fill({{dW1, (size_t)d * K * 2}, {dW2, (size_t)2 * F * d * 2}, {dg, (size_t)d * 4},
+                      {dWdown, (size_t)d * F * 2}},
+                     stream);
+  }
   if (!dOut || !X || !W1 || !H || !r || !AB || !Y || !g || !W2 || !Wdown || !dX || !dR || !dW1 || !dW2 || !dg ||
       !dWdown || !ws)
     return CODA_ERR_INVALID_ARG;
@@ -921,8 +1004,8 @@ namespace coda {
 namespace {
 coda_status check_rope(const void* X, const void* W, int M, int d, int n_q, int n_kv, int head_dim, int seq_len,
                        float base) {
-  if (!X || !W) return CODA_ERR_INVALID_ARG;
-  if (M < 1 || d < 1 || n_q < 1 || n_kv < 1 || seq_len < 1 || !(base > 1.f)) return CODA_ERR_INVALID_ARG;
+  if (!W || (M > 0 && !X)) return CODA_ERR_INVALID_ARG;
+  if (M < 0 || d < 1 || n_q < 1 || n_kv < 1 || seq_len < 1 || !(base > 1.f)) return CODA_ERR_INVALID_ARG;
   if (d % 64 != 0 || !(head_dim == 64 || head_dim == 128 || head_dim == 256)) return CODA_ERR_UNSUPPORTED_SHAPE;
   return CODA_OK;
 }
@@ -935,6 +1018,7 @@ extern "C" {
 coda_status coda_qkv_rope_fwd(const void* X, const void* Wqkv, void* QKV, int M, int d, int n_q, int n_kv,
                               int head_dim, int seq_len, float base, void* ws, size_t ws_bytes, void* stream) {
   CODA_TRY(check_rope(X, Wqkv, M, d, n_q, n_kv, head_dim, seq_len, base));
+  if (M == 0) return CODA_OK;  // empty batch
   if (!QKV || !ws) return CODA_ERR_INVALID_ARG;
   const void* ptrs[] = {X, Wqkv, QKV, ws};
   for (const void* q : ptrs)
@@ -969,6 +1053,7 @@ coda_status coda_qkv_rope_bwd(const void* dQKV, const void* X, const void* Wqkv,
                               int n_q, int n_kv, int head_dim, int seq_len, float base, void* ws, size_t ws_bytes,
                               void* stream) {
   CODA_TRY(check_rope(X, Wqkv, M, d, n_q, n_kv, head_dim, seq_len, base));
+  if (M == 0) return zero_fill({{dW, (size_t)(n_q + 2 * n_kv) * head_dim * d * 2}}, stream);  // empty batch
   if (!dQKV || !dX || !dW || !ws) return CODA_ERR_INVALID_ARG;
   const void* ptrs[] = {dQKV, X, Wqkv, dX, dW, ws};
   for (const void* q : ptrs)
@@ -1003,6 +1088,7 @@ size_t coda_grg_fwd_unfused_workspace_bytes(int M, int K, int d, int N) {
 coda_status coda_grg_fwd_unfused(const void* X, const void* W1, const void* R, const void* g, const void* W2,
                                  void* H, float* r, void* Y, void* AB, void* U, int M, int K, int d, int N,
                                  float eps, void* ws, size_t ws_bytes, void* stream) {
+  if (M == 0) return !(eps > 0.f) ? CODA_ERR_INVALID_ARG : check_grg_shapes(1, K, d, N);  // empty batch
   if (!X || !W1 || !R || !g || !W2 || !H || !r || !Y || !AB || !U || !ws) return CODA_ERR_INVALID_ARG;
   if (!(eps > 0.f)) return CODA_ERR_INVALID_ARG;
   CODA_TRY(check_grg_shapes(M, K, d, N));
@@ -1039,6 +1125,10 @@ coda_status coda_grg_bwd_unfused(const void* dY, const void* dH_in_or_null, cons
                                  const void* H, const float* r, const void* AB, const void* U, const void* g,
                                  const void* W2, void* dX, void* dR, void* dW1, void* dW2, float* dg, int M, int K,
                                  int d, int N, void* ws, size_t ws_bytes, void* stream) {
+  if (M == 0) {  // empty batch: zero weight gradients
+    CODA_TRY(check_grg_shapes(1, K, d, N));
+    return zero_fill({{dW1, (size_t)d * K * 2}, {dW2, (size_t)N * d * 2}, {dg, (size_t)d * 4}}, stream);
+  }
   if (!dY || !X || !W1 || !H || !r || !AB || !U || !g || !W2 || !dX || !dR || !dW1 || !dW2 || !dg || !ws)
     return CODA_ERR_INVALID_ARG;
   CODA_TRY(check_grg_shapes(M, K, d, N));
@@ -1081,6 +1171,7 @@ extern "C" {
 
 coda_status coda_swiglu_fwd_unfused(const void* X, const void* Wgu, const void* Wdown, void* Y, void* AB, void* Out,
                                     int M, int d, int F, void* ws, size_t ws_bytes, void* stream) {
+  if (M == 0) return check_swiglu_shapes(1, d, F);  // empty batch
   if (!X || !Wgu || !Wdown || !Y || !AB || !Out || !ws) return CODA_ERR_INVALID_ARG;
   CODA_TRY(check_swiglu_shapes(M, d, F));
   const void* ptrs[] = {X, Wgu, Wdown, Y, AB, Out, ws};
@@ -1106,6 +1197,10 @@ size_t coda_swiglu_bwd_unfused_workspace_bytes(int M, int d, int F) {
 coda_status coda_swiglu_bwd_unfused(const void* dOut, const void* X, const void* Wgu, const void* Wdown,
                                     const void* Y, const void* AB, void* dX, void* dWgu, void* dWdown, int M, int d,
                                     int F, void* ws, size_t ws_bytes, void* stream) {
+  if (M == 0) {  // empty batch: zero weight gradients
+    CODA_TRY(check_swiglu_shapes(1, d, F));
+    return zero_fill({{dWgu, (size_t)2 * F * d * 2}, {dWdown, (size_t)d * F * 2}}, stream);
+  }
   if (!dOut || !X || !Wgu || !Wdown || !Y || !AB || !dX || !dWgu || !dWdown || !ws) return CODA_ERR_INVALID_ARG;
   CODA_TRY(check_swiglu_shapes(M, d, F));
   const void* ptrs[] = {dOut, X, Wgu, Wdown, Y, AB, dX, dWgu, dWdown, ws};
@@ -1159,6 +1254,7 @@ coda_status static_scratch(int dev, void** out) {
 extern "C" coda_status coda_grg_fwd_prefolded_static(const void* X, const void* W1, const void* R, const void* W2g,
                                                      void* H, float* r, void* Y, void* AB_or_null, int M, int K,
                                                      int d, int N, float eps, void* stream) {
+  if (M == 0) return !(eps > 0.f) ? CODA_ERR_INVALID_ARG : check_grg_shapes(1, K, d, N);  // empty batch
   if (!X || !W1 || !R || !W2g || !H || !r || !Y) return CODA_ERR_INVALID_ARG;
   if (!(eps > 0.f)) return CODA_ERR_INVALID_ARG;
   CODA_TRY(check_grg_shapes(M, K, d, N));

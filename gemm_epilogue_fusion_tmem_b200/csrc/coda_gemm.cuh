@@ -115,6 +115,22 @@ __device__ __forceinline__ void load32_bf16(const __nv_bfloat16* p, bool valid, 
   }
 }
 
+// One thread's 32 bf16 of a row-major input chunk, held packed in registers
+// so it can be loaded one chunk ahead of its use (and, for a tile's first
+// chunk, before the accumulator is ready): the epilogue's per-row inputs
+// (residual, H, dH_in, saved a/b) then arrive while earlier work runs.
+struct Pref32 {
+  uint4 q[4];
+};
+__device__ __forceinline__ void pref_load(Pref32& x, const __nv_bfloat16* p, bool valid) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) x.q[j] = valid ? ldg_nc_v4(p + 8 * j) : make_uint4(0u, 0u, 0u, 0u);
+}
+__device__ __forceinline__ void pref_unpack(const Pref32& x, float (&f)[32]) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) unpack8(x.q[j], f + 8 * j);
+}
+
 // Per-warp tile store through shared memory: the warp's 32 rows x 32 columns
 // of one output go to a 2 KiB staging tile (64-byte rows, 16-byte chunks
 // swizzled by (row >> 1) & 3, which makes the row-per-thread writes
@@ -192,12 +208,30 @@ __device__ __forceinline__ void warp_column_sums(float (&v)[32], int lane) {
 }
 
 
+// Loads the first chunk of a tile's per-row epilogue inputs (issued before the
+// wait for the accumulator).
+template <int EPI>
+__device__ __forceinline__ void epilogue_prefetch(const GemmParams& p, int row, bool rv, int n_blk, Pref32& x0,
+                                                  Pref32& x1) {
+  if constexpr (EPI == EPI_RESID_RMS || EPI == EPI_DN) {
+    const size_t off = (size_t)row * p.ld_in0 + (size_t)n_blk * BN;
+    pref_load(x0, p.in0 + off, rv);
+    if constexpr (EPI == EPI_DN) {
+      if (p.in1 != nullptr) pref_load(x1, p.in1 + (size_t)row * p.ldo + (size_t)n_blk * BN, rv);
+    }
+  } else if constexpr (EPI == EPI_SWIGLU_BWD) {
+    const __nv_bfloat16* ab = p.in0 + (size_t)row * p.ld_in0 + (size_t)n_blk * BN;
+    pref_load(x0, ab, rv);
+    pref_load(x1, ab + p.split, rv);
+  }
+}
+
 // One 128-row half-tile of the epilogue: this thread owns output row `row`
 // (valid when rv), `group32` = (row - lane) / 32 indexes the per-warp partials.
 template <int EPI>
 __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbase, int row, bool rv, int group32,
                                               int n_blk, int lane, EpiStore& es, const CUtensorMap* mo1,
-                                              const CUtensorMap* mo2) {
+                                              const CUtensorMap* mo2, Pref32& x0, Pref32& x1) {
   if constexpr (EPI == EPI_STORE) {
     const int n0 = n_blk * BN;
 #pragma unroll 1
@@ -222,7 +256,8 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbas
     for (int c = 0; c < BN; c += 32) {
       if (n0 + c >= p.N) break;
       float rres[32];
-      load32_bf16(p.in0 + (size_t)row * p.ld_in0 + n0 + c, rv, rres);
+      pref_unpack(x0, rres);
+      if (c + 32 < BN && n0 + c + 32 < p.N) pref_load(x0, p.in0 + (size_t)row * p.ld_in0 + n0 + c + 32, rv);
       float v[32];
       tmem_ld32(tbase + c, v);
       uint4 hq[4];
@@ -281,8 +316,10 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbas
 #pragma unroll 1
     for (int c = 0; c < BN; c += 32) {
       if (n0 + c >= p.N) break;
+      const bool more = c + 32 < BN && n0 + c + 32 < p.N;
       float h[32];
-      load32_bf16(p.in0 + (size_t)row * p.ld_in0 + n0 + c, rv, h);
+      pref_unpack(x0, h);
+      if (more) pref_load(x0, p.in0 + (size_t)row * p.ld_in0 + n0 + c + 32, rv);
       float v[32];
       tmem_ld32(tbase + c, v);
       float g[32];
@@ -292,7 +329,8 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbas
       for (int i = 0; i < 32; ++i) o[i] = fmaf(g[i], v[i], -cc * h[i]);
       if (p.in1 != nullptr) {
         float e[32];
-        load32_bf16(p.in1 + (size_t)row * p.ldo + n0 + c, rv, e);
+        pref_unpack(x1, e);
+        if (more) pref_load(x1, p.in1 + (size_t)row * p.ldo + n0 + c + 32, rv);
 #pragma unroll
         for (int i = 0; i < 32; ++i) o[i] += e[i];
       }
@@ -396,9 +434,13 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbas
     for (int c = 0; c < BN; c += 32) {
       if (n0 + c >= p.N) break;
       float a[32], b[32];
-      const __nv_bfloat16* ab = p.in0 + (size_t)row * p.ld_in0 + n0 + c;
-      load32_bf16(ab, rv, a);
-      load32_bf16(ab + p.split, rv, b);
+      pref_unpack(x0, a);
+      pref_unpack(x1, b);
+      if (c + 32 < BN && n0 + c + 32 < p.N) {
+        const __nv_bfloat16* ab = p.in0 + (size_t)row * p.ld_in0 + n0 + c + 32;
+        pref_load(x0, ab, rv);
+        pref_load(x1, ab + p.split, rv);
+      }
       float dy[32];
       tmem_ld32(tbase + c, dy);
 #pragma unroll
@@ -644,14 +686,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int tile = first_tile; tile < num_tiles; tile += tile_step) {
       int m_blk, n_blk;
       tile_coords(tile, p.num_m_tiles, p.num_n_tiles, p.group_m, m_blk, n_blk);
+      const int row0 = m_blk * C::TILE_M + (int)rank * 128 + q * 32;
+      Pref32 x0, x1;
+      epilogue_prefetch<EPI>(p, row0 + lane, row0 + lane < p.M, n_blk, x0, x1);
       // Warp-uniform outcome: tcgen05.ld below needs all 32 lanes converged.
       const bool ok = mbar_wait(&tfull[acc], acc_phase, ctl, 2 + q, kWaitAccFull);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
-      const int row0 = m_blk * C::TILE_M + (int)rank * 128 + q * 32;
       es.row0 = row0;
-      epilogue_tile<EPI>(p, tbase, row0 + lane, row0 + lane < p.M, row0 / 32, n_blk, lane, es, &tmO1, &tmO2);
+      epilogue_tile<EPI>(p, tbase, row0 + lane, row0 + lane < p.M, row0 / 32, n_blk, lane, es, &tmO1, &tmO2, x0,
+                         x1);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {

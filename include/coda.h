@@ -37,6 +37,12 @@
  *    alignment, device capability, launch failures).  Device-side errors are
  *    read with coda_status_query().  No call aborts or throws.
  *  - Requires an sm_100 device (B200); otherwise CODA_ERR_NO_SM100.
+ *  - An empty batch (M = 0 tokens) is valid everywhere: the other sizes are
+ *    still checked, no kernel runs, and row-sized pointers may be NULL.  A
+ *    forward call then writes nothing; a backward call writes its weight
+ *    gradients (dW1, dW2, dg, dWgu, dWdown, dW) as zeros, the sum over no rows,
+ *    on `stream`.  coda_gemm with M = 0 or N = 0 does nothing; with K = 0 it
+ *    writes C = 0.  Negative sizes return CODA_ERR_INVALID_ARG.
  */
 #ifndef CODA_H_
 #define CODA_H_
@@ -50,7 +56,7 @@ extern "C" {
 
 typedef enum {
   CODA_OK = 0,
-  CODA_ERR_INVALID_ARG = 1,         /* null pointer, non-positive size, eps <= 0 */
+  CODA_ERR_INVALID_ARG = 1,         /* null pointer, negative or zero weight size, eps <= 0 */
   CODA_ERR_UNSUPPORTED_SHAPE = 2,   /* a dimension violates the stated multiple */
   CODA_ERR_MISALIGNED = 3,          /* a pointer is not 16-byte aligned */
   CODA_ERR_WORKSPACE_TOO_SMALL = 4, /* ws_bytes below the *_workspace_bytes() size */
@@ -91,15 +97,19 @@ void coda_set_wait_limit_ns(uint64_t ns);
 coda_status coda_selftest_wait_timeout(void* ws, uint64_t limit_ns, void* stream);
 
 /* Kernel timing hook.  Arms a one-shot pair of CUDA events around the next
- * launch, from the calling host thread, of a GEMM whose epilogue is
- * `epilogue` (one of CODA_EPI_*), whichever entry point makes it: ev_start is
- * recorded on that launch's stream immediately before the kernel and ev_stop
- * immediately after, then the hook disarms itself.  ev_start and ev_stop are
- * cudaEvent_t handles created and owned by the caller (timing enabled); the
- * library only records them.  Both NULL disarms.  Returns CODA_ERR_INVALID_ARG
- * for an unknown epilogue or a single NULL event.  Recording the events takes
- * the place of the programmatic (PDL) overlap between that kernel and its
- * neighbours, so an armed launch can start a few microseconds later. */
+ * launch, from the calling host thread, of the kernel `kernel` names, whichever
+ * entry point makes it: a GEMM by its epilogue (CODA_EPI_*) or a light pass
+ * (CODA_KERNEL_*).  ev_start is recorded on that launch's stream immediately
+ * before the kernel and ev_stop immediately after; then that pair disarms.
+ * Up to 16 pairs may be armed at once; several pairs armed for the same kernel
+ * fire on its successive launches, in arming order (e.g. the three plain-store
+ * GEMMs of the block's backward).  ev_start and ev_stop are cudaEvent_t handles
+ * created and owned by the caller (timing enabled); the library only records
+ * them.  Both NULL disarms every pair of this thread.  Returns
+ * CODA_ERR_INVALID_ARG for an unknown kernel id, a single NULL event or a full
+ * table.  Recording the events takes the place of the programmatic (PDL)
+ * overlap at that kernel's two boundaries, so an armed launch can start a few
+ * microseconds later. */
 #define CODA_EPI_STORE 0      /* plain store (optional column scale) */
 #define CODA_EPI_RESID_RMS 1  /* + residual, H, partial sums of squares */
 #define CODA_EPI_SWIGLU 2     /* r scaling + SwiGLU (the gate/up GEMM) */
@@ -108,7 +118,14 @@ coda_status coda_selftest_wait_timeout(void* ws, uint64_t limit_ns, void* stream
 #define CODA_EPI_XENT 5       /* online max / sum-exp (the logits GEMM) */
 #define CODA_EPI_XENT_BWD 6   /* softmax - one-hot, dlogits */
 #define CODA_EPI_ROPE 7       /* rotary embedding (the QKV GEMM) */
-coda_status coda_profile_arm(int epilogue, void* ev_start, void* ev_stop);
+#define CODA_KERNEL_FOLD_GAIN 16          /* W2g = W2 diag(g) */
+#define CODA_KERNEL_RMS_ROWREDUCE 17      /* r from the partial sums of squares */
+#define CODA_KERNEL_SWIGLU_BWD_ROWSTAT 18 /* dA' = r [da | db] and the row coefficient c */
+#define CODA_KERNEL_COL_REDUCE 19         /* dg from its column partials */
+#define CODA_KERNEL_ROWCOEF_REDUCE 20     /* c from its row partials (MLP block backward) */
+#define CODA_KERNEL_XENT_REDUCE 21        /* loss and log-sum-exp from the tile partials */
+#define CODA_KERNEL_ROPE_UNROTATE 22      /* inverse rotation of dQ, dK (RoPE backward) */
+coda_status coda_profile_arm(int kernel, void* ev_start, void* ev_stop);
 
 /* ---------------------------------------------------------------- building block */
 
@@ -160,7 +177,7 @@ size_t coda_grg_fwd_workspace_bytes(int M, int K, int d, int N, int prefolded);
  *          W2g_or_null: optional caller-folded diag(g)-scaled W2 [N, d]; when
  *          null the fold runs inside this call into the workspace.
  * Outputs: H [M,d] bf16, r [M] fp32, Y [M,F] bf16, AB_or_null [M,N] bf16.
- * Requires M >= 1, K % 64 == 0, d % 64 == 0, N % 128 == 0 (F % 64 == 0), eps > 0.
+ * Requires M >= 0, K % 64 == 0, d % 64 == 0, N % 128 == 0 (F % 64 == 0), eps > 0.
  * Rows, the last partial-RMS tile and the last F tile may be ragged. */
 coda_status coda_grg_fwd(const void* X, const void* W1, const void* R, const void* g,
                          const void* W2, const void* W2g_or_null,
@@ -224,7 +241,7 @@ size_t coda_swiglu_fwd_workspace_bytes(int M, int d, int F);
  *   gate/up GEMM + epilogue: A = X Wgu^T;  Y = silu(a) * b;  AB = [a | b]
  *   down GEMM:               Out = Y Wdown^T
  * Inputs X [M,d], Wgu [2F,d], Wdown [d,F].  Outputs Y [M,F], AB_or_null
- * [M,2F], Out [M,d] (bf16).  Requires M >= 1, d % 64 == 0, F % 64 == 0. */
+ * [M,2F], Out [M,d] (bf16).  Requires M >= 0, d % 64 == 0, F % 64 == 0. */
 coda_status coda_swiglu_fwd(const void* X, const void* Wgu, const void* Wdown,
                             void* Y, void* AB_or_null, void* Out,
                             int M, int d, int F, void* ws, size_t ws_bytes, void* stream);
@@ -293,7 +310,7 @@ size_t coda_xent_fwd_workspace_bytes(int M, int d, int V);
  *   lse_i = log sum_j exp(logits_ij),  loss_i = lse_i - logits_i,t_i.
  * Inputs X [M,d] bf16, W [V,d] bf16, targets [M] int32 in [0, V).
  * Outputs loss [M] and lse [M] fp32 (loss is NaN for an out-of-range target).
- * Requires M >= 1, d % 64 == 0, V % 64 == 0.  Logits are fp32 accumulators. */
+ * Requires M >= 0, d % 64 == 0, V % 64 == 0.  Logits are fp32 accumulators. */
 coda_status coda_xent_fwd(const void* X, const void* W, const int32_t* targets, float* loss, float* lse,
                           int M, int d, int V, void* ws, size_t ws_bytes, void* stream);
 

@@ -80,3 +80,30 @@ def test_argument_errors_return_before_any_device_work(lib):
     assert lib.coda_grg_fwd(*([one] * 10), 128, 64, 64, 128, 0.0, one, 1 << 20, None) == 1
     # d must be a multiple of 64
     assert lib.coda_grg_fwd(*([one] * 10), 128, 64, 96, 128, 1e-6, one, 1 << 20, None) == 2
+
+
+def test_empty_batch_and_negative_sizes_on_the_host(lib):
+    """M = 0 is a valid empty batch: forward calls return OK without touching a
+    device (row pointers may be NULL); a backward call needs its weight-gradient
+    pointers; negative sizes are invalid."""
+    P = ctypes.c_void_p
+    one = P(256)
+    lib.coda_grg_fwd.argtypes = [P] * 10 + [ctypes.c_int] * 4 + [ctypes.c_float, P, ctypes.c_size_t, P]
+    nulls = [None, one, None, one, one, None, None, None, None, None]  # X, W1, R, g, W2, W2g, H, r, Y, AB
+    assert lib.coda_grg_fwd(*nulls, 0, 64, 64, 128, 1e-6, None, 0, None) == 0
+    assert lib.coda_grg_fwd(*nulls, 0, 64, 96, 128, 1e-6, None, 0, None) == 2   # d still checked
+    assert lib.coda_grg_fwd(*nulls, 0, 64, 64, 128, 0.0, None, 0, None) == 1    # eps still checked
+    assert lib.coda_grg_fwd(*nulls, -1, 64, 64, 128, 1e-6, None, 0, None) == 1
+    lib.coda_grg_bwd.argtypes = [P] * 9 + [P] * 5 + [ctypes.c_int] * 4 + [P, ctypes.c_size_t, P]
+    # dY, dH_in, X, W1, H, r, AB, g, W2 | dX, dR, dW1 (NULL), dW2, dg
+    args = [None, None, None, one, None, None, None, one, one, None, None, None, one, one]
+    assert lib.coda_grg_bwd(*args, 0, 64, 64, 128, None, 0, None) == 1
+    lib.coda_gemm.argtypes = [P, P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                              P, ctypes.c_size_t, P]
+    assert lib.coda_gemm(None, None, None, 0, 128, 64, 0, 0, None, 0, None) == 0
+    assert lib.coda_gemm(None, None, None, 128, 0, 64, 0, 0, None, 0, None) == 0
+    assert lib.coda_gemm(one, one, one, -5, 128, 64, 0, 0, one, 256, None) == 1
+    assert lib.coda_gemm(None, None, None, 128, 128, 0, 0, 0, None, 0, None) == 1  # K = 0 writes C: needs C
+    lib.coda_swiglu_fwd.argtypes = [P] * 6 + [ctypes.c_int] * 3 + [P, ctypes.c_size_t, P]
+    assert lib.coda_swiglu_fwd(None, one, one, None, None, None, 0, 64, 64, None, 0, None) == 0
+    assert lib.coda_swiglu_fwd(None, one, one, None, None, None, 0, 64, 100, None, 0, None) == 2

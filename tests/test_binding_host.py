@@ -50,13 +50,22 @@ def test_status_strings_round_trip():
 
 
 def test_profile_hook_argument_checks():
-    """coda_profile_arm validates its arguments without touching the GPU."""
+    """coda_profile_arm validates its arguments and its table without touching the GPU."""
     import ctypes
     lib = B.library()
-    fake = ctypes.c_void_p(1)  # never recorded: every call below is refused or disarms
-    assert lib.coda_profile_arm(99, fake, fake) == B.CODA_ERR_INVALID_ARG
-    assert lib.coda_profile_arm(-1, fake, fake) == B.CODA_ERR_INVALID_ARG
-    assert lib.coda_profile_arm(B.EPI_SWIGLU, fake, None) == B.CODA_ERR_INVALID_ARG
-    assert lib.coda_profile_arm(B.EPI_SWIGLU, None, fake) == B.CODA_ERR_INVALID_ARG
-    assert lib.coda_profile_arm(B.EPI_SWIGLU, None, None) == 0  # disarm
-    assert (B.EPI_STORE, B.EPI_SWIGLU, B.EPI_XENT, B.EPI_ROPE) == (0, 2, 5, 7)
+    fake = ctypes.c_void_p(1)  # never recorded: nothing is launched in this process
+    try:
+        for bad in (-1, 8, 15, 23, 99):
+            assert lib.coda_profile_arm(bad, fake, fake) == B.CODA_ERR_INVALID_ARG, bad
+        assert lib.coda_profile_arm(B.EPI_SWIGLU, fake, None) == B.CODA_ERR_INVALID_ARG
+        assert lib.coda_profile_arm(B.EPI_SWIGLU, None, fake) == B.CODA_ERR_INVALID_ARG
+        ids = list(range(8)) + list(range(16, 23))
+        for k in ids:
+            assert lib.coda_profile_arm(k, fake, fake) == 0, k
+        assert lib.coda_profile_arm(B.EPI_STORE, fake, fake) == 0  # 16th pair: the table is full
+        assert lib.coda_profile_arm(B.EPI_STORE, fake, fake) == B.CODA_ERR_INVALID_ARG
+    finally:
+        assert lib.coda_profile_arm(0, None, None) == 0  # disarm all
+    assert lib.coda_profile_arm(B.EPI_STORE, fake, fake) == 0  # room again after disarming
+    assert lib.coda_profile_arm(0, None, None) == 0
+    assert (B.EPI_STORE, B.EPI_SWIGLU, B.EPI_ROPE, B.KERNEL_FOLD_GAIN, B.KERNEL_ROPE_UNROTATE) == (0, 2, 7, 16, 22)

@@ -76,3 +76,29 @@ def test_profile_hook_times_one_launch(cuda_lib):
     assert flops / (k / 1e3) < 3.0e15  # below any B200 bf16 rate: the pair spans the kernel
     assert after > 0.5 * k, (k, after)
     B.profile_arm(B.EPI_SWIGLU)
+
+
+def test_profile_hook_times_every_kernel_of_a_step(cuda_lib):
+    """Pairs armed for all ten kernels of the block's forward and backward fire
+    once each, in launch order (three for the plain-store GEMMs), and bracket
+    non-overlapping stretches of the stream."""
+    B = cuda_lib
+    M, K, d, F = 1024, 1024, 1024, 2048
+    t = synth.grg_inputs(M, K, d, F, seed=12)
+    dv = {k: v.cuda() for k, v in t.items()}
+    ids = [B.KERNEL_FOLD_GAIN, B.EPI_RESID_RMS, B.KERNEL_RMS_ROWREDUCE, B.EPI_SWIGLU,
+           B.KERNEL_SWIGLU_BWD_ROWSTAT, B.EPI_DN, B.KERNEL_COL_REDUCE, B.EPI_STORE, B.EPI_STORE, B.EPI_STORE]
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in ids]
+    fo = B.grg_fwd(dv["X"], dv["W1"], dv["R"], dv["g"], dv["W2"], 1e-6)  # warm: allocations, tensor maps
+    bo = B.grg_bwd(dv["dY"], dv["X"], dv["W1"], fo["H"], fo["r"], fo["AB"], dv["g"], dv["W2"])
+    torch.cuda.synchronize()
+    for k, (x, y) in zip(ids, ev):
+        B.profile_arm(k, x, y)
+    B.grg_fwd(dv["X"], dv["W1"], dv["R"], dv["g"], dv["W2"], 1e-6, out=fo)
+    B.grg_bwd(dv["dY"], dv["X"], dv["W1"], fo["H"], fo["r"], fo["AB"], dv["g"], dv["W2"], out=bo)
+    torch.cuda.synchronize()
+    B.profile_arm(0)
+    for i, (x, y) in enumerate(ev):
+        assert x.elapsed_time(y) > 0.0, i
+        if i + 1 < len(ev):
+            assert y.elapsed_time(ev[i + 1][0]) >= 0.0, i
