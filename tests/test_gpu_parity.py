@@ -166,6 +166,31 @@ def test_grg_structured_exact_indexing(cuda_lib):
         assert not np.any(a), "only the one-hot entry may be nonzero"
 
 
+def test_grg_zero_rows_forward_backward(cuda_lib):
+    """Tokens whose X and R rows are zero: H = 0 there, so RMSNorm's degenerate
+    case r = 1/sqrt(eps) applies, a = b = Y = 0, and the backward gives dA' = 0,
+    dH = dR = 0 and dX = 0 in those rows, exactly.  Every output also matches
+    the oracle at the usual tolerance."""
+    M, K, d, F, eps = 256, 512, 512, 1024, 1e-6
+    t = synth.grg_inputs(M, K, d, F, seed=13)
+    zero = [0, 77, 255]
+    t["X"][zero] = 0
+    t["R"][zero] = 0
+    td = _cuda(t)
+    o = cuda_lib.grg_fwd(td["X"], td["W1"], td["R"], td["g"], td["W2"], eps)
+    b = cuda_lib.grg_bwd(td["dY"], td["X"], td["W1"], o["H"], o["r"], o["AB"], td["g"], td["W2"])
+    torch.cuda.synchronize()
+    fwd, bwd, fwd_s, bwd_s = _grg_oracle(t, eps)
+    _check_fwd(o, fwd, fwd_s, "grg_fwd zero rows")
+    for k in ("dX", "dR", "dW1", "dW2", "dg"):
+        assert_tol(b[k], bwd_s[k], f"grg_bwd zero rows {k}", outlier_frac=BWD_OUTLIER_FRAC)
+        assert_pure(b[k], bwd[k], f"grg_bwd zero rows {k}")
+    r = o["r"].cpu().numpy()
+    np.testing.assert_allclose(r[zero], 1.0 / np.sqrt(eps), rtol=1e-6)
+    for name, v in (("H", o["H"]), ("Y", o["Y"]), ("AB", o["AB"]), ("dX", b["dX"]), ("dR", b["dR"])):
+        assert torch.count_nonzero(v[zero]).item() == 0, name
+
+
 # ----------------------------------------------------------------------------- SwiGLU MLP
 
 SWIGLU_CASES = [

@@ -85,6 +85,30 @@ def test_constant_rows_closed_form_r():
         np.testing.assert_allclose(f["r"], 1.0 / np.sqrt(c * c + eps), rtol=1e-14)
 
 
+def test_zero_rows_degenerate_case():
+    """A row with X_i = 0 and R_i = 0 has H_i = 0: r_i = 1/sqrt(eps) exactly
+    (the RMSNorm degenerate case), Y_i = 0, and its gradients dH_i = dX_i = 0
+    (a = b = 0 makes da = db = 0).  The other rows are unaffected: they equal
+    the oracle run on those rows alone (rows are independent), and the weight
+    gradients get nothing from the zero row."""
+    rng = np.random.default_rng(21)
+    M, K, d, F, eps = 4, 6, 8, 5, 1e-4
+    X, R = rng.standard_normal((M, K)), rng.standard_normal((M, d))
+    X[2], R[2] = 0.0, 0.0
+    W1, W2 = rng.standard_normal((d, K)), rng.standard_normal((2 * F, d))
+    g, dY = 1 + 0.1 * rng.standard_normal(d), rng.standard_normal((M, F))
+    f = O.grg_forward(X, W1, R, g, W2, eps)
+    b = O.grg_backward(dY, X, W1, R, g, W2, eps, fwd=f)
+    assert f["r"][2] == 1.0 / math.sqrt(eps)
+    assert not np.any(f["Y"][2]) and not np.any(b["dX"][2]) and not np.any(b["dR"][2])
+    keep = [0, 1, 3]
+    f3 = O.grg_forward(X[keep], W1, R[keep], g, W2, eps)
+    b3 = O.grg_backward(dY[keep], X[keep], W1, R[keep], g, W2, eps, fwd=f3)
+    np.testing.assert_allclose(f["Y"][keep], f3["Y"], rtol=1e-13, atol=1e-13)
+    for k in ("dW1", "dW2", "dg"):
+        np.testing.assert_allclose(b[k], b3[k], rtol=1e-12, atol=1e-12)
+
+
 def test_unit_rms_rows_when_gain_is_one():
     """g = 1: mean_j n_ij^2 = ms_i / (ms_i + eps); exactly 1 at eps = 0."""
     rng = np.random.default_rng(2)
