@@ -456,7 +456,7 @@ def _make_unfused_step(kind, s, bwd, dev):
 def _time_loop(fn, steps, warmup, device, world, barrier):
     """Device time of `steps` calls of fn (CUDA events on the current stream), max over ranks."""
     import torch
-    for _ in range(max(warmup, 3)):
+    for _ in range(max(warmup, 3) if warmup is not None else 0):
         fn()
     torch.cuda.synchronize()
     st = torch.cuda.current_stream()
@@ -469,6 +469,22 @@ def _time_loop(fn, steps, warmup, device, world, barrier):
     torch.cuda.synchronize()
     barrier()
     return max_over_ranks(e0.elapsed_time(e1), device, world)
+
+
+def _time_interleaved(fa, fb, steps, warmup, device, world, barrier, rounds=6):
+    """Median ms per call of fa and of fb, timed in alternating bursts (fa, fb,
+    fa, fb, ...) so that both see the same thermal and power-cap drift; each
+    burst is max over ranks."""
+    import statistics
+    per = max(1, steps // rounds)
+    for _ in range(max(warmup, 3)):
+        fa()
+        fb()
+    ta, tb = [], []
+    for _ in range(rounds):
+        ta.append(_time_loop(fa, per, None, device, world, barrier) / per)
+        tb.append(_time_loop(fb, per, None, device, world, barrier) / per)
+    return statistics.median(ta), statistics.median(tb)
 
 
 def _grg_kernels(s, bwd):
@@ -709,19 +725,11 @@ def run_coda(a):
                 B.grg_bwd(dev["dY"], dev["X"], dev["W1"], hf["H"], hf["r"], hf["AB"], dev["g"], dev["W2"], out=hb,
                           ws=hws)
 
-        for _ in range(max(a.warmup, 3)):
-            hstep()
-        torch.cuda.synchronize()
-        barrier()
-        e0.record(st)
-        for _ in range(a.steps):
-            hstep()
-        e1.record(st)
-        torch.cuda.synchronize()
-        barrier()
-        h_ms = max_over_ranks(e0.elapsed_time(e1), device, world)
-        variants["activation_gain"] = {"ms_per_step": round(h_ms / a.steps, 4),
-                                       "value": round(replica_throughput(flops, a.steps, world, h_ms), 2),
+        f_ms, h_ms = _time_interleaved(step, hstep, a.steps, a.warmup, device, world, barrier)
+        variants["activation_gain"] = {"ms_per_step": round(h_ms, 4),
+                                       "value": round(replica_throughput(flops, 1, world, h_ms), 2),
+                                       "fused_ms_per_step": round(f_ms, 4),
+                                       "timing": "alternating bursts with the folded-gain step, medians",
                                        "what": "coda_grg_fwd_hg: GEMM1 stores H*g, GEMM2 reads W2 unfolded"}
         del hws
 
@@ -731,20 +739,22 @@ def run_coda(a):
     unfused = None
     if kind in ("grg", "swiglu") and not a.no_unfused:
         ustep, ulaunch, uws = _make_unfused_step(kind, s, bwd, dev)
-        u_ms = _time_loop(ustep, a.steps, a.warmup, device, world, barrier)
-        unfused = {"ms_per_step": round(u_ms / a.steps, 4),
-                   "value": round(replica_throughput(flops, a.steps, world, u_ms), 2), "unit": "TFLOP/s",
-                   "fused_speedup": round(u_ms / ms_max, 4), "gpu_launches_per_step": ulaunch,
+        # Fused and unfused in alternating bursts (medians), so drift under the
+        # power cap does not favour whichever runs first.
+        f_ms, u_ms = _time_interleaved(step, ustep, a.steps, a.warmup, device, world, barrier)
+        unfused = {"ms_per_step": round(u_ms, 4),
+                   "value": round(replica_throughput(flops, 1, world, u_ms), 2), "unit": "TFLOP/s",
+                   "fused_ms_per_step": round(f_ms, 4), "fused_speedup": round(u_ms / f_ms, 4),
+                   "gpu_launches_per_step": ulaunch, "timing": "alternating bursts of fused and unfused steps, "
+                                                               "median ms per step of each",
                    "what": "same GEMM kernels with plain stores; residual add, RMSNorm, SwiGLU and their backward "
                            "as separate HBM-round-trip kernels"}
         for dname in ("fwd", "bwd"):
             ff, uf = getattr(step, dname, None), getattr(ustep, dname, None)
             if ff is None or uf is None:
                 continue
-            f_ms = _time_loop(ff, a.steps, a.warmup, device, world, barrier)
-            un_ms = _time_loop(uf, a.steps, a.warmup, device, world, barrier)
-            unfused[dname] = {"fused_ms": round(f_ms / a.steps, 4), "unfused_ms": round(un_ms / a.steps, 4),
-                              "speedup": round(un_ms / f_ms, 4)}
+            fd, ud = _time_interleaved(ff, uf, a.steps, a.warmup, device, world, barrier)
+            unfused[dname] = {"fused_ms": round(fd, 4), "unfused_ms": round(ud, 4), "speedup": round(ud / fd, 4)}
         del uws
 
     # Roofline of the dominant kernel: its average launch duration inside the

@@ -12,19 +12,37 @@ namespace coda {
 // toolin.ai five-primitive table lists the RMSNorm weight broadcast as a
 // vector-load primitive; folding it once per weight update removes it from
 // the epilogue entirely).
+constexpr int FOLD_UNROLL = 4;  // independent 16-byte loads in flight per thread
 __global__ void fold_gain_kernel(const __nv_bfloat16* __restrict__ W2, const __nv_bfloat16* __restrict__ g,
                                  __nv_bfloat16* __restrict__ W2g, int d, long long n_vec8) {
   griddep_wait();
-  const long long stride = (long long)gridDim.x * blockDim.x;
-  for (long long v = (long long)blockIdx.x * blockDim.x + threadIdx.x; v < n_vec8; v += stride) {
-    const long long e = v * 8;
-    const int j = (int)(e % d);
-    float w[8], gg[8];
-    unpack8(ldg_nc_v4(W2 + e), w);
-    unpack8(ldg_nc_v4(g + j), gg);
+  const int dv = d / 8;  // 8-element vectors per row
+  const long long S = (long long)gridDim.x * blockDim.x;
+  const int s_mod = (int)(S % dv);
+  long long v = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  int jv = (int)(v % dv);  // column vector of v; advanced by S mod dv per step
+  for (; v < n_vec8; v += FOLD_UNROLL * S) {
+    uint4 w[FOLD_UNROLL];
+    int jj[FOLD_UNROLL];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) w[i] *= gg[i];
-    stg_v4(W2g + e, pack8(w));
+    for (int u = 0; u < FOLD_UNROLL; ++u) {
+      const long long vu = v + u * S;
+      jj[u] = jv;
+      if (vu < n_vec8) w[u] = ldg_nc_v4(W2 + vu * 8);
+      jv += s_mod;
+      if (jv >= dv) jv -= dv;
+    }
+#pragma unroll
+    for (int u = 0; u < FOLD_UNROLL; ++u) {
+      const long long vu = v + u * S;
+      if (vu >= n_vec8) break;
+      float f[8], gg[8];
+      unpack8(w[u], f);
+      unpack8(ldg_nc_v4(g + jj[u] * 8), gg);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) f[i] *= gg[i];
+      stg_v4(W2g + vu * 8, pack8(f));
+    }
   }
 }
 

@@ -113,6 +113,21 @@ def test_grg_forward_prefolded_weight(cuda_lib):
     _check_fwd(o, fwd, fwd_s, "grg_fwd prefolded")
 
 
+@pytest.mark.parametrize("N,d", [(384, 192), (8192, 1024), (2, 4096)])
+def test_fold_gain_bit_exact(cuda_lib, N, d):
+    """W2g = bf16(W2 * g): the fp32 product of two bf16 values is exact, so the
+    only rounding is the final round-to-nearest-even, and the kernel must match
+    the oracle's rounding of the exact product bit for bit (sizes with a ragged
+    last grid-stride step, several steps, and fewer vectors than threads)."""
+    gen = torch.Generator().manual_seed(N + d)
+    W2 = torch.randn(N, d, generator=gen).to(torch.bfloat16)
+    g = (1 + 0.1 * torch.randn(d, generator=gen)).to(torch.bfloat16)
+    W2g = cuda_lib.fold_gain(W2.cuda(), g.cuda())
+    torch.cuda.synchronize()
+    ref = O.round_bf16(f64(W2) * f64(g)[None, :])
+    np.testing.assert_array_equal(f64(W2g), ref)
+
+
 @pytest.mark.parametrize("with_dH_in", [False, True])
 @pytest.mark.parametrize("M,K,d,F,eps", GRG_CASES)
 def test_grg_backward(cuda_lib, M, K, d, F, eps, with_dH_in):
