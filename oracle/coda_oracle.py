@@ -26,7 +26,7 @@ Sources (the pages give no formulas; see each function for the reading taken):
 * toolin.ai §実験結果 and kucoin (ru) §Результаты эксперимента: the backward of
   GEMM-Residual-PartialRMS-GEMM and of SwiGLU are the measured kernels.
 
-Readings taken where the pages are silent (all listed in the design doc):
+Readings taken where the pages are silent:
 eps sits inside the root, r_i = 1/sqrt(mean_j H_ij^2 + eps), the mean runs over
 the full hidden width d; the first F rows of the gate/up weight are the gate
 (silu input) and the last F the up projection; weights use the [out, in]
