@@ -755,6 +755,26 @@ def run_coda(a):
                                        "what": "coda_grg_fwd_hg: GEMM1 stores H*g, GEMM2 reads W2 unfolded"}
         del hws
 
+    # The same step captured once in a CUDA graph and replayed (no per-launch
+    # host overhead), timed in alternating bursts with the eager step.
+    try:
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(graph, stream=side):
+                step()
+        torch.cuda.current_stream().wait_stream(side)
+        e_ms, g_ms = _time_interleaved(step, graph.replay, a.steps, a.warmup, device, world, barrier)
+        variants["cuda_graph"] = {"ms_per_step": round(g_ms, 4),
+                                  "value": round(replica_throughput(flops, 1, world, g_ms), 2),
+                                  "eager_ms_per_step": round(e_ms, 4),
+                                  "timing": "alternating bursts with the eager step, medians",
+                                  "what": "the same step captured once with torch.cuda.graph and replayed"}
+        del graph
+    except RuntimeError as err:  # capture not possible: report it instead of a number
+        variants["cuda_graph"] = {"error": str(err)[:200]}
+
     # The unfused comparison sequence, timed the same way right after, and
     # both paths split into forward and backward (the pages compare each
     # direction separately).
