@@ -91,7 +91,7 @@ def _describe(name, kind, s, bwd):
         what = f"full MLP block (GEMM-Residual-RMSNorm-GEMM-SwiGLU + down projection + residual) {name} fwd+bwd"
     else:
         what = "SwiGLU MLP fwd+bwd"
-    return {"workload": what, **s, "global_batch": s["M"]}
+    return {"workload": what, **s, "tokens": s["M"]}
 
 
 # ----------------------------------------------------------------------------- CPU oracle timing
