@@ -7,7 +7,7 @@ partial RMS, the row reduce, GEMM2 + r + SwiGLU, and (fwd+bwd workloads) the
 SwiGLU backward + row statistic, the dn GEMM, the dg column reduce, the dW2,
 dX and dW1 GEMMs.  All of it runs in libcoda.so through the C ABI.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 7B|70B|1B|swiglu|tiny]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 7B|70B|1B|swiglu|tiny|xent|rope|block7B]
   python bench.py --impl reference ...   (the fp64 CPU oracle on the host cores)
 
 Prints one JSON line on rank 0.  Under torchrun each rank runs an independent
