@@ -107,3 +107,46 @@ def test_empty_batch_and_negative_sizes_on_the_host(lib):
     lib.coda_swiglu_fwd.argtypes = [P] * 6 + [ctypes.c_int] * 3 + [P, ctypes.c_size_t, P]
     assert lib.coda_swiglu_fwd(None, one, one, None, None, None, 0, 64, 64, None, 0, None) == 0
     assert lib.coda_swiglu_fwd(None, one, one, None, None, None, 0, 64, 100, None, 0, None) == 2
+
+
+C_CONSUMER = r"""
+#include "coda.h"
+#include <stdio.h>
+int main(void) {
+  /* host-only calls: no device is touched */
+  printf("%d\n", coda_version());
+  printf("%s\n", coda_status_string(CODA_ERR_WORKSPACE_TOO_SMALL));
+  printf("%zu\n", coda_grg_fwd_workspace_bytes(8192, 4096, 4096, 22016, 0));
+  printf("%zu\n", coda_grg_bwd_workspace_bytes(8192, 4096, 4096, 22016));
+  printf("%d\n", (int)coda_grg_fwd(0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 256, 512, 512, 2048, 1e-6f, 0, 0, 0));
+  printf("%d\n", (int)coda_profile_arm(99, 0, 0));
+  return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_links_from_c(lib, tmp_path):
+    """include/coda.h compiles as strict C11 and a C program links against
+    libcoda.so and gets the same answers as the Python binding."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not available")
+    from gemm_epilogue_fusion_tmem_b200 import build as Bld
+    src = tmp_path / "consumer.c"
+    src.write_text(C_CONSUMER)
+    exe = tmp_path / "consumer"
+    libdir = os.path.dirname(Bld.LIB_PATH)
+    subprocess.run([gcc, "-std=c11", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", Bld.INCLUDE, str(src),
+                    "-L", libdir, "-lcoda", f"-Wl,-rpath,{libdir}", "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split("\n")
+    lib.coda_status_string.restype = ctypes.c_char_p
+    for f in (lib.coda_grg_fwd_workspace_bytes, lib.coda_grg_bwd_workspace_bytes):
+        f.restype = ctypes.c_size_t
+    assert int(out[0]) == lib.coda_version()
+    assert out[1] == lib.coda_status_string(4).decode()
+    assert int(out[2]) == lib.coda_grg_fwd_workspace_bytes(8192, 4096, 4096, 22016, 0)
+    assert int(out[3]) == lib.coda_grg_bwd_workspace_bytes(8192, 4096, 4096, 22016)
+    assert int(out[4]) == 1  # null pointers: CODA_ERR_INVALID_ARG before any device work
+    assert int(out[5]) == 1  # unknown kernel id
