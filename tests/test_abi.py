@@ -119,7 +119,7 @@ int main(void) {
   printf("%zu\n", coda_grg_fwd_workspace_bytes(8192, 4096, 4096, 22016, 0));
   printf("%zu\n", coda_grg_bwd_workspace_bytes(8192, 4096, 4096, 22016));
   printf("%d\n", (int)coda_grg_fwd(0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 256, 512, 512, 2048, 1e-6f, 0, 0, 0));
-  printf("%d\n", (int)coda_profile_arm(99, 0, 0));
+  printf("%d\n", (int)coda_profile_arm(99, (void*)16, (void*)16));
   return 0;
 }
 """
