@@ -2,22 +2,30 @@
 //
 // GEMM-epilogue structure (toolin.ai CODA article, section 核心の洞察; kucoin.com
 // (ru) CODA article, section «В «Финале» спрятаны сокровища»): a fixed mainloop
-// computes a 128 x 256 fp32 tile into tensor memory, and an epilogue transforms
-// the tile while it is still on chip before anything reaches HBM.  The
-// epilogue variants are built from the pages' primitives (five-primitive
-// table): elementwise transforms (residual add, SwiGLU, its backward),
-// vector loads (r, c, g), matrix-tile loads/stores (R, H, a/b, outputs) and
-// tile-wise reductions (row sums of squares, column sums for dg).
+// computes an fp32 tile into tensor memory, and an epilogue transforms the
+// tile while it is still on chip before anything reaches HBM.  The epilogue
+// variants are built from the pages' primitives (five-primitive table):
+// elementwise transforms (residual add, SwiGLU, its backward, RoPE), vector
+// loads (r, c, g), matrix-tile loads/stores (R, H, a/b, outputs), tile-wise
+// reductions (row sums of squares, column sums for dg) and, for the
+// cross-entropy, the stateful online max / sum-exp.
+//
+// Tiles: by default a CTA pair (cluster of 2, tcgen05 cta_group::2) computes a
+// 256 x 256 tile, each CTA holding 128 rows of A and half of B; with PAIR =
+// false one CTA computes 128 x 256.
 //
 // Roles (192 threads, one CTA per SM):
 //   warp 0      TMA producer (one lane): 128B-swizzled K-major or MN-major
 //               operand tiles into a STAGES-deep shared-memory ring.
-//   warp 1      TMEM owner and MMA issuer (one lane): tcgen05.mma kind::f16,
-//               M=128 N=256 K=16, into one of two TMEM accumulators
-//               (2 x 256 columns), commit -> mbarriers.
+//   warp 1      TMEM owner and MMA issuer (one lane of the pair's leader):
+//               tcgen05.mma kind::f16, K=16, into one of two TMEM
+//               accumulators (2 x 256 columns), commits -> mbarriers.
 //   warps 2-5   epilogue: tcgen05.ld 32 lanes x 32 columns per step, one
-//               output row per thread, 16-byte global stores.
+//               output row per thread; outputs staged in shared memory and
+//               written with TMA tile stores.
 // The two TMEM accumulators let tile i's epilogue overlap tile i+1's mainloop.
+// Every wait is bounded (see mbar_wait); a role that gives up records the
+// failure in the status word and the CTA drains and exits.
 #pragma once
 
 #include "coda_ptx.cuh"
