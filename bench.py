@@ -884,8 +884,10 @@ def run_reference(a):
     t0 = time.perf_counter()
     _oracle_step(kind, s, bwd, inputs, probe)
     rate = _flops(kind, dict(s, M=probe), bwd) / max(time.perf_counter() - t0, 1e-3)
-    # Each step a sample sized for about 2 s so the whole run stays within a few minutes.
-    rows = max(probe, min(s["M"], int(2.0 * rate / _flops(kind, dict(s, M=1), bwd))))
+    # Each step a sample sized for about 2 s (less when many steps are asked
+    # for) so the whole run stays within about two minutes.
+    per_step_s = min(2.0, 120.0 / max(1, a.steps + a.warmup))
+    rows = max(probe, min(s["M"], int(per_step_s * rate / _flops(kind, dict(s, M=1), bwd))))
     for _ in range(a.warmup):
         _oracle_step(kind, s, bwd, inputs, rows)
     t0 = time.perf_counter()
