@@ -69,3 +69,40 @@ def test_profile_hook_argument_checks():
     assert lib.coda_profile_arm(B.EPI_STORE, fake, fake) == 0  # room again after disarming
     assert lib.coda_profile_arm(0, None, None) == 0
     assert (B.EPI_STORE, B.EPI_SWIGLU, B.EPI_ROPE, B.KERNEL_FOLD_GAIN, B.KERNEL_ROPE_UNROTATE) == (0, 2, 7, 16, 22)
+
+
+def test_oracle_and_product_path_share_no_code():
+    """The package never imports the oracle and the oracle never imports the
+    package (only the seeded input generator, which holds none of the method's
+    arithmetic, is shared through the tests); bench.py touches the oracle only
+    inside its CPU legs."""
+    import ast
+    import os
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    pkg = os.path.join(root, "gemm_epilogue_fusion_tmem_b200")
+
+    def imports(path):
+        tree = ast.parse(open(path, encoding="utf-8").read())
+        out = []
+        for node in ast.walk(tree):
+            if isinstance(node, ast.Import):
+                out += [a.name for a in node.names]
+            elif isinstance(node, ast.ImportFrom) and node.module:
+                out.append(node.module)
+        return out
+
+    for name in os.listdir(pkg):
+        if name.endswith(".py"):
+            assert not any(m.split(".")[0] == "oracle" for m in imports(os.path.join(pkg, name))), name
+    for name in os.listdir(os.path.join(root, "oracle")):
+        if name.endswith(".py"):
+            mods = imports(os.path.join(root, "oracle", name))
+            assert not any(m.startswith("gemm_epilogue_fusion_tmem_b200") for m in mods), name
+            assert not any(m in ("torch", "ctypes") for m in mods), name
+    # bench.py: oracle imports only inside the CPU-leg functions
+    tree = ast.parse(open(os.path.join(root, "bench.py"), encoding="utf-8").read())
+    for fn in [n for n in tree.body if isinstance(n, ast.FunctionDef)]:
+        uses = any(isinstance(x, ast.ImportFrom) and x.module and x.module.startswith("oracle") for x in ast.walk(fn))
+        if uses:
+            assert fn.name in ("_oracle_step", "_oracle_inputs", "cpu_baseline", "run_reference"), fn.name
+    assert not any(isinstance(x, (ast.Import, ast.ImportFrom)) and "oracle" in ast.dump(x) for x in tree.body)
