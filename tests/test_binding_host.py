@@ -5,6 +5,8 @@ before anything reaches the library's compute entry points, and every entry
 point the binding names is exported by the built library.
 """
 
+import os
+
 import pytest
 import torch
 
@@ -106,3 +108,20 @@ def test_oracle_and_product_path_share_no_code():
         if uses:
             assert fn.name in ("_oracle_step", "_oracle_inputs", "cpu_baseline", "run_reference"), fn.name
     assert not any(isinstance(x, (ast.Import, ast.ImportFrom)) and "oracle" in ast.dump(x) for x in tree.body)
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    """Without the built CUDA library the binding raises; there is no fallback."""
+    import subprocess
+    import sys
+    code = (
+        "import sys; sys.path.insert(0, %r)\n"
+        "from gemm_epilogue_fusion_tmem_b200 import binding as B\n"
+        "B.LIB_PATH = %r\n"
+        "try:\n"
+        "    B.library()\n"
+        "except RuntimeError as e:\n"
+        "    print('raised', 'not built' in str(e))\n"
+    ) % (os.path.dirname(os.path.dirname(os.path.abspath(__file__))), str(tmp_path / "absent.so"))
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=120).stdout
+    assert out.strip() == "raised True", out
