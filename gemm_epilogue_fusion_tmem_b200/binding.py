@@ -95,8 +95,36 @@ def library() -> ctypes.CDLL:
             fn = getattr(lib, name)
             fn.restype = res
             fn.argtypes = args
+            if name not in _UNRANGED and not name.endswith("_workspace_bytes"):
+                setattr(lib, name, _Ranged(fn, name))
         _lib = lib
         return lib
+
+
+# Host-side entry points that enqueue no GPU work get no NVTX range.
+_UNRANGED = {"coda_status_string", "coda_version", "coda_set_wait_limit_ns", "coda_profile_arm",
+             "coda_status_query"}
+
+
+class _Ranged:
+    """A C entry point called inside an NVTX range of its own name, so profilers
+    (ncu --nvtx, Nsight Systems) attribute each call's kernels to it.  Without
+    a profiler attached the push and pop do nothing."""
+
+    __slots__ = ("_fn", "_name")
+
+    def __init__(self, fn, name):
+        self._fn, self._name = fn, name
+
+    def __call__(self, *args):
+        torch.cuda.nvtx.range_push(self._name)
+        try:
+            return self._fn(*args)
+        finally:
+            torch.cuda.nvtx.range_pop()
+
+    def __getattr__(self, key):
+        return getattr(self._fn, key)
 
 
 def _status_string(status: int) -> str:
