@@ -5,7 +5,8 @@ checks tensor dtypes/devices/contiguity, allocates outputs and the workspace
 with torch (device memory and streams are all torch is used for), and passes
 raw device pointers plus ``torch.cuda.current_stream()`` to the C entry points
 of the same names.  There is no CPU fallback: if the library is missing or the
-device is not sm_100, calls raise.
+device is not sm_100, calls raise.  Each call into an entry point that enqueues
+GPU work is wrapped in an NVTX range of the entry point's name.
 """
 
 from __future__ import annotations
