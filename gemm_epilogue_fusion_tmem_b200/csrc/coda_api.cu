@@ -57,7 +57,8 @@ struct DevInfo {
   bool configured[kKernelSlots] = {};
   int max_clusters[kKernelSlots] = {};
 };
-DevInfo g_dev[64];
+constexpr int kMaxDevices = 64;  // device ordinals the per-device tables cover
+DevInfo g_dev[kMaxDevices];
 
 int g_last_sms = 148;
 int num_sms() { return g_last_sms; }
@@ -65,7 +66,7 @@ int num_sms() { return g_last_sms; }
 inline int ew_grid(long long n_vec8) { return (int)std::min<long long>(cdiv(n_vec8, 256), (long long)num_sms() * 16); }
 
 coda_status current_device(int& dev) {
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return CODA_ERR_CUDA;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return CODA_ERR_CUDA;
   DevInfo& di = g_dev[dev];
   if (di.num_sms == 0) {
     int sms = 0, major = 0;
@@ -1237,9 +1238,10 @@ namespace coda {
 namespace {
 constexpr size_t kStaticScratchBytes = kStatusBytes + (size_t)CODA_STATIC_PARTIALS_MAX * sizeof(float);
 __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
-std::atomic<void*> g_static_scratch_addr[64];
+std::atomic<void*> g_static_scratch_addr[kMaxDevices];
 
 coda_status static_scratch(int dev, void** out) {
+  if (dev < 0 || dev >= kMaxDevices) return CODA_ERR_CUDA;
   void* p = g_static_scratch_addr[dev].load();
   if (p == nullptr) {
     if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) return CODA_ERR_CUDA;
@@ -1291,4 +1293,16 @@ extern "C" coda_status coda_grg_fwd_prefolded_static(const void* X, const void* 
   CODA_TRY(launch_status(launch_ex(rms_rowreduce_kernel, dim3(cdiv(M, 256)), dim3(256), 0, s, 1, (const float*)P, T,
                                    r, M, 1.0f / (float)d, eps)));
   return gemm_swiglu(H, W2g, r, Y, AB_or_null, M, d, F, scratch, s);
+}
+
+extern "C" coda_status coda_static_status_query(void* stream, uint32_t* detail) {
+  int dev;
+  CODA_TRY(current_device(dev));
+  void* scratch = nullptr;
+  CODA_TRY(static_scratch(dev, &scratch));
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return CODA_ERR_CUDA;
+  uint32_t w[2] = {0, 0};
+  if (cudaMemcpy(w, scratch, sizeof(w), cudaMemcpyDeviceToHost) != cudaSuccess) return CODA_ERR_CUDA;
+  if (detail != nullptr) *detail = w[1];
+  return static_cast<coda_status>(w[0]);
 }

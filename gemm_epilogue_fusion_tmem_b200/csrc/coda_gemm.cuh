@@ -42,7 +42,7 @@ constexpr uint32_t TMEM_COLS = 2 * BN;
 
 enum Epi : int {
   EPI_STORE = 0,       // out = bf16(acc [* g_col])
-  EPI_RESID_RMS = 1,   // H = bf16(acc + R); P[row, ntile] = sum bf16(H)^2; optional Hg = bf16(H*g)
+  EPI_RESID_RMS = 1,   // H = bf16(acc + R); P[row, ntile] = sum H^2; optional Hg = bf16(H*g) (H the stored bf16)
   EPI_SWIGLU = 2,      // a = r*acc_gate, b = r*acc_up; Y = silu(a)*b; AB = [a|b]
   EPI_DN = 3,          // dH = g*acc - c*H (+dH_in); column partials of acc*H
   EPI_SWIGLU_BWD = 4,  // dY = acc; da, db from a, b; dA = [da|db] (optionally r-scaled, with c partials)
@@ -275,19 +275,20 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbas
 #pragma unroll
         for (int i = 0; i < 8; ++i) h[i] = v[8 * j + i] + rres[8 * j + i];
         hq[j] = pack8(h);
-        float hb[8];
-        unpack8(hq[j], hb);  // square the stored (bf16-rounded) H
+        unpack8(hq[j], v + 8 * j);  // v now holds the stored (bf16-rounded) H
 #pragma unroll
-        for (int i = 0; i < 8; ++i) ss = fmaf(hb[i], hb[i], ss);
+        for (int i = 0; i < 8; ++i) ss = fmaf(v[8 * j + i], v[8 * j + i], ss);
       }
       es.begin();
       es.put_packed(hq, mo1, n0 + c);
       if (p.out2 != nullptr) {
-        // Activation-side gain: Hg = bf16(H * g), the second GEMM's operand.
+        // Activation-side gain: Hg = bf16(H * g) from the stored H, the second
+        // GEMM's operand (the product of two bf16 values is exact in fp32, so
+        // the only rounding is the final one).
         float g[32];
         load32_bf16(p.colvec + n0 + c, true, g);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) g[i] *= v[i] + rres[i];
+        for (int i = 0; i < 32; ++i) g[i] *= v[i];
         es.put(g, mo2, n0 + c);
       }
       es.flush();

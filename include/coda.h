@@ -432,12 +432,20 @@ coda_status coda_swiglu_bwd_unfused(const void* dOut, const void* X, const void*
  *    partial sums are fully overwritten); calls whose work overlaps on the GPU
  *    (different streams, or host threads without ordering) race on the array,
  *    so callers must serialise them.
- *  - A device-side wait timeout is recorded in that internal status word,
- *    which callers cannot read; use coda_grg_fwd with a workspace when the
- *    device status must be observable. */
+ *  - A device-side wait timeout is recorded in that internal status word;
+ *    coda_static_status_query reads it back. */
 coda_status coda_grg_fwd_prefolded_static(const void* X, const void* W1, const void* R, const void* W2g,
                                           void* H, float* r, void* Y, void* AB_or_null,
                                           int M, int K, int d, int N, float eps, void* stream);
+
+/* Status of the last coda_grg_fwd_prefolded_static call on the current
+ * device: synchronises `stream`, copies the static scratch's status word to
+ * the host and returns it (CODA_OK, or CODA_ERR_DEVICE_TIMEOUT with the
+ * kernel / role / reason word in *detail when detail is not NULL).  The word
+ * is zeroed at the start of every such call.  Allocates nothing; like the
+ * first forward call it looks the array's address up on first use.  Returns
+ * CODA_ERR_CUDA when the stream cannot be synchronised or the copy fails. */
+coda_status coda_static_status_query(void* stream, uint32_t* detail);
 
 #ifdef __cplusplus
 }

@@ -222,15 +222,39 @@ def swiglu_backward(dOut, X, Wgu, Wdown, fwd: dict | None = None) -> dict:
 
 # ----------------------------------------------------------------------------- storage precision
 #
-# The method keeps every tensor it hands from one pass to the next in HBM as
-# bf16: GEMM1's epilogue stores H and GEMM2 reads it back (toolin.ai
-# §核心の洞察; kucoin (ru) §«В «Финале» спрятаны сокровища»: H goes to memory, r is
-# deferred to GEMM2's epilogue), the saved activations of the matrix-tile
-# store primitive (five-primitive table) are bf16, and every GEMM consumes
-# bf16 operands.  The *_stored functions below evaluate the same definitions
-# in float64 but round each stored tensor with ``store`` (default: round to
-# nearest bf16, ties to even) at the point where the method stores it.  With
-# ``store=lambda x: x`` they reduce to the textbook functions above (pinned).
+# The same definitions evaluated at the precision of the method's dataflow:
+# every tensor that crosses HBM between two GEMM-epilogue programs is bf16
+# there, so the functions below round (with ``store``, default round to
+# nearest bf16, ties to even) exactly those tensors and nothing else.  Which
+# tensors those are follows from the pages, not from any kernel:
+#
+# (S1) A GEMM's operands are bf16 tensors in HBM.  In the forward these are
+#      H, which GEMM1's epilogue stores and GEMM2 reads back (toolin.ai
+#      §核心の洞察 and kucoin (ru) §«В «Финале» спрятаны сокровища»: H goes to
+#      memory, the RMSNorm scale r does not), the gain-folded weight
+#      W2g = bf16(diag(g) W2) (the fold of the RMSNorm gain into the second
+#      GEMM's weight), or, with the gain on the activation side, Hg, and in the
+#      MLP the down projection's operand Y.
+# (S2) The saved activations a and b are stored for the backward (the
+#      matrix-tile store primitive, "saving activations for the backward", in
+#      the five-primitive table of both pages).
+# (S3) The backward of a GEMM-epilogue program is again a GEMM with an
+#      epilogue (kucoin (ru) §«В «Финале» спрятаны сокровища»: a block-local
+#      forward epilogue gives a backward of the same structure).  Its GEMMs are
+#      the adjoint of the forward GEMM, and the operand they read is the
+#      gradient at the forward GEMM's raw output, before that GEMM's epilogue
+#      transform.  GEMM2's epilogue applies r (the pages defer r to it), so
+#      GEMM2's adjoint reads dZ = diag(r) dA, the gradient of Z = H W2g^T with
+#      A = diag(r) Z; GEMM1's epilogue adds the residual, so GEMM1's adjoint
+#      reads dH (which is the output dR, stored bf16); the MLP's gate/up GEMM
+#      has no row scale, so its adjoint reads dA itself.
+#
+# Everything else stays float64: r, the SwiGLU output Y computed from the
+# unrounded a and b, the RMSNorm backward's row term.  With store = identity
+# every function here reduces to the textbook one above (pinned), and the
+# placement of each rounding is pinned by hand-derived cases in
+# tests/golden/ (a value of H on a bf16 midpoint, a pre-activation on a
+# midpoint, a row scale r = 1/3 that moves the rounding of dZ).
 
 
 def round_bf16(x) -> np.ndarray:
@@ -251,28 +275,28 @@ def _ident(x):
 
 
 def grg_forward_stored(X, W1, R, g, W2, eps: float, store=round_bf16, gain: str = "weight") -> dict:
-    """grg_forward with the method's dataflow at storage precision.
+    """grg_forward at the precision of the method's dataflow (S1, S2 above).
 
-      H   = store(X W1^T + R)                  stored by GEMM1, read by the rest
-      r   = 1/sqrt(mean_j H_ij^2 + eps)        from the stored H
-      gain = "weight":     W2g = store(W2 diag(g)),  A = diag(r) (H W2g^T)
-      gain = "activation": Hg = store((X W1^T + R) diag(g)), A = diag(r) (Hg W2^T)
-                                               r deferred past GEMM2 (the pages' identity)
-      a, b = A[:, :F], A[:, F:];  Y = silu(a) * b   (Y from the unrounded a, b)
-      a_s, b_s = store(a), store(b)            saved for the backward
+      H    = store(X W1^T + R)                 GEMM1's epilogue stores H (S1)
+      r    = 1/sqrt(mean_j H_ij^2 + eps)       from the H that GEMM2 reads
+      gain = "weight":     Z = H W2g^T,  W2g = store(W2 diag(g))      (S1, the fold)
+      gain = "activation": Z = Hg W2^T,  Hg  = store(H diag(g))       (S1, gain on H)
+      A    = diag(r) Z                         r applied after GEMM2 (the pages' identity)
+      a, b = A[:, :F], A[:, F:];  Y = silu(a) * b      (from the unrounded a, b)
+      a_s, b_s = store(a), store(b)            saved for the backward (S2)
     """
     X, W1, R, g, W2 = map(_f64, (X, W1, R, g, W2))
-    H_exact = X @ W1.T + R
-    H = store(H_exact)
+    H = store(X @ W1.T + R)
     d = H.shape[1]
     ms = np.sum(H * H, axis=1) / d
     r = 1.0 / np.sqrt(ms + eps)
     if gain == "weight":
-        A = r[:, None] * (H @ store(W2 * g[None, :]).T)
+        Z = H @ store(W2 * g[None, :]).T
     elif gain == "activation":
-        A = r[:, None] * (store(H_exact * g[None, :]) @ W2.T)
+        Z = store(H * g[None, :]) @ W2.T
     else:
         raise ValueError(f"gain must be 'weight' or 'activation', got {gain!r}")
+    A = r[:, None] * Z
     F = W2.shape[0] // 2
     a, b = A[:, :F], A[:, F:]
     Y = silu(a) * b
@@ -281,10 +305,15 @@ def grg_forward_stored(X, W1, R, g, W2, eps: float, store=round_bf16, gain: str 
 
 def grg_backward_stored(dY, X, W1, R, g, W2, eps: float, dH_in=None, store=round_bf16,
                         fwd: dict | None = None) -> dict:
-    """grg_backward at storage precision: the same chain rule, fed by the stored
-    forward tensors (H, a, b), with the SwiGLU gradient stored once in units of
-    r_i ([da | db] scaled by the row's r, the operand of the two GEMMs that
-    consume it) and dH stored before the dX / dW1 GEMMs read it.
+    """grg_backward at the precision of the method's dataflow (S2, S3 above).
+
+    The chain rule of grg_backward, fed by the stored H and the saved a_s, b_s,
+    with two bf16 operands on the way:
+      dA  = [da | db] from SwiGLU at (dY, a_s, b_s)
+      dZ  = store(diag(r) dA)              gradient at GEMM2's raw output (S3)
+      dW2 = g * (dZ^T H);  du = dZ W2 / r;  dg = sum_i du * n;  dn = du * g
+      dH  = r dn - (r^3/d)(sum_k dn H) H (+ dH_in);   dR = dH
+      dX  = store(dR) W1;  dW1 = store(dR)^T X   GEMM1's adjoint reads the stored dR (S3)
     """
     if fwd is None:
         fwd = grg_forward_stored(X, W1, R, g, W2, eps, store)
@@ -294,8 +323,8 @@ def grg_backward_stored(dY, X, W1, R, g, W2, eps: float, dH_in=None, store=round
     n = H * r[:, None]
     u = n * g[None, :]
     da, db = _swiglu_grads(dY, a, b)
-    dA = np.concatenate([da, db], axis=1)
-    dA = store(dA * r[:, None]) / r[:, None]
+    dZ = store(np.concatenate([da, db], axis=1) * r[:, None])
+    dA = dZ / r[:, None]                  # the stored operand in units of the textbook dA
     dW2 = dA.T @ u
     du = dA @ W2
     dg = np.sum(du * n, axis=0)
@@ -304,12 +333,13 @@ def grg_backward_stored(dY, X, W1, R, g, W2, eps: float, dH_in=None, store=round
     dH = dn * r[:, None] + (dr * (-0.5) * r ** 3)[:, None] * (2.0 / d) * H
     if dH_in is not None:
         dH = dH + _f64(dH_in)
-    dHs = store(dH)
-    return {"dA": dA, "dH": dH, "dR": dH, "dX": dHs @ W1, "dW1": dHs.T @ X, "dW2": dW2, "dg": dg}
+    dRs = store(dH)
+    return {"dZ": dZ, "dA": dA, "dH": dH, "dR": dH, "dX": dRs @ W1, "dW1": dRs.T @ X, "dW2": dW2, "dg": dg}
 
 
 def swiglu_forward_stored(X, Wgu, Wdown, store=round_bf16) -> dict:
-    """swiglu_forward with Y stored before the down GEMM and a, b saved stored."""
+    """swiglu_forward with the down projection reading the stored Y (S1) and
+    a, b saved stored (S2)."""
     X, Wgu, Wdown = map(_f64, (X, Wgu, Wdown))
     A = X @ Wgu.T
     F = Wgu.shape[0] // 2
@@ -320,8 +350,8 @@ def swiglu_forward_stored(X, Wgu, Wdown, store=round_bf16) -> dict:
 
 
 def swiglu_backward_stored(dOut, X, Wgu, Wdown, store=round_bf16, fwd: dict | None = None) -> dict:
-    """swiglu_backward fed by the stored Y, a, b, with [da | db] stored before
-    the dWgu / dX GEMMs read it."""
+    """swiglu_backward fed by the stored Y, a, b, with the gate/up GEMM's
+    adjoint reading the stored gradient at its output, dA = [da | db] (S3)."""
     if fwd is None:
         fwd = swiglu_forward_stored(X, Wgu, Wdown, store)
     dOut, X, Wgu, Wdown = map(_f64, (dOut, X, Wgu, Wdown))

@@ -1,3 +1,4 @@
+import json
 import os
 import sys
 
@@ -21,3 +22,20 @@ def cuda_lib():
         pytest.skip("no CUDA device")
     from gemm_epilogue_fusion_tmem_b200 import binding
     return binding
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """Worst |err| / bound and the count above the bound of every parity check run."""
+    from tests.parity import REPORT
+    if not REPORT:
+        return
+    tr = terminalreporter
+    tr.section("parity: worst |err| / bound per check (above_bound must be 0)")
+    for rec in REPORT:
+        tr.write_line(f"{rec['worst_ratio']:8.4f}  above={rec['above_bound']:<4d} n={rec['n']:<10d} "
+                      f"[{rec['kind']}] {rec['check']}")
+    path = os.environ.get("CODA_PARITY_REPORT")
+    if path:
+        with open(path, "a") as f:
+            for rec in REPORT:
+                f.write(json.dumps(rec) + "\n")

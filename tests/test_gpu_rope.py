@@ -4,7 +4,8 @@ The rotation angles are computed in fp32 on the GPU (pos * 2^(j * k)), as
 common LLaMA implementations do; at positions below 2^13 the angle error is
 below 1e-3 rad, so the bf16 bound |gpu - ref| <= 1e-2 |ref| + 1e-2 rms(ref)
 holds against the fp64 angles of the oracle.  The backward's stored operand
-(the inverse-rotated gradient) is bf16, compared like the block's gradients.
+(the inverse-rotated gradient) is bf16, compared like the block's gradients:
+against pure fp64 the bound is widened by the deviation its rounding produces.
 """
 
 import pytest
@@ -12,6 +13,7 @@ import torch
 
 from gemm_epilogue_fusion_tmem_b200 import synth
 from oracle import coda_oracle as O
+from tests import error_model as E
 from tests.parity import assert_pure, assert_tol, f64
 
 pytestmark = pytest.mark.gpu
@@ -38,6 +40,8 @@ def test_qkv_rope_forward_backward(cuda_lib, M, d, nq, nkv, hd, S, base):
     assert_tol(Q, f["QKV"], f"{tag} QKV")
     bs = O.qkv_rope_backward(dQ, X, W, nq, nkv, hd, S, base, store=O.round_bf16)
     b0 = O.qkv_rope_backward(dQ, X, W, nq, nkv, hd, S, base)
+    assert_pure(Q, f["QKV"], f"{tag} QKV")
+    sg = E.sigma(E.stored_operand_var(b0["dpre"], X, W))
     for k in ("dX", "dW"):
         assert_tol(b[k], bs[k], f"{tag} {k}")
-        assert_pure(b[k], b0[k], f"{tag} {k}")
+        assert_pure(b[k], b0[k], f"{tag} {k}", sg[k])

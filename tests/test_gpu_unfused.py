@@ -1,8 +1,9 @@
 """The unfused comparison sequence, and the fused path's error against it.
 
 The unfused calls run the block operator by operator (every intermediate in
-HBM).  They are checked against the pure fp64 oracle within the bound derived
-from bf16 storage, and the fused path's error must be comparable or smaller:
+HBM).  They are checked against the pure fp64 oracle within the stated bound
+widened by the deviation their own bf16 intermediates produce
+(tests/error_model.py), and the fused path's error must be comparable or smaller:
 the pages report the reparameterisation's numerical error as comparable to the
 PyTorch reference and sometimes smaller, thanks to the mainloop's fp32
 accumulator (kucoin.com (ru) CODA article, section «Результаты эксперимента»).
@@ -16,6 +17,7 @@ import torch
 
 from gemm_epilogue_fusion_tmem_b200 import synth
 from oracle import coda_oracle as O
+from tests import error_model as E
 from tests.parity import assert_pure, f64
 
 pytestmark = pytest.mark.gpu
@@ -50,8 +52,9 @@ def test_unfused_matches_oracle_and_fused_error_is_comparable(cuda_lib, M, K, d,
     unf = {"H": uf["H"], "Y": uf["Y"], "a": uf["AB"][:, :F], "b": uf["AB"][:, F:], **ub}
     fus = {"H": fu["H"], "Y": fu["Y"], "a": fu["AB"][:, :F], "b": fu["AB"][:, F:], **bu}
     ref = {**{k: fwd[k] for k in ("H", "Y", "a", "b")}, **{k: bwd[k] for k in ("dX", "dR", "dW1", "dW2", "dg")}}
+    sg = E.sigma(E.grg_unfused_var(fwd, bwd, X, W1, g, W2, dY))
     for k, v in unf.items():
-        assert_pure(v, ref[k], f"unfused {tag} {k}")
+        assert_pure(v, ref[k], f"unfused {tag} {k}", sg[k])
     np.testing.assert_allclose(f64(uf["r"]), fwd["r"], rtol=1e-3)
     for k in ref:
         e_f, e_u = _rms_err(fus[k], ref[k]), _rms_err(unf[k], ref[k])
@@ -75,8 +78,9 @@ def test_swiglu_unfused_matches_oracle_and_fused_error_is_comparable(cuda_lib, M
     unf = {"Y": uo["Y"], "Out": uo["Out"], **ub}
     fus = {"Y": fo["Y"], "Out": fo["Out"], **fb}
     tag = f"swiglu M={M} d={d} F={F}"
+    sg = E.sigma(E.swiglu_unfused_var(fwd, bwd, X, Wgu, Wdown, dOut))
     for k, v in unf.items():
-        assert_pure(v, ref[k], f"unfused {tag} {k}")
+        assert_pure(v, ref[k], f"unfused {tag} {k}", sg[k])
     for k in ref:
         e_f, e_u = _rms_err(fus[k], ref[k]), _rms_err(unf[k], ref[k])
         rms = float(np.sqrt(np.mean(ref[k] ** 2)))

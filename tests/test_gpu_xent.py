@@ -3,8 +3,9 @@
 loss and lse are fp32 results of fp32-accumulated logits: |gpu - ref| <=
 1e-4 |ref| + 1e-4 (fp32 accumulation over d bf16 products and fp32 exp/log
 give errors near 1e-6; the bound leaves two orders of margin).  dX and dW come
-from bf16-stored dlogits: the bf16 bound against the storage-precision oracle
-and the derived bound against pure fp64, as for the block.
+from bf16-stored dlogits: the bf16 bound against the storage-precision oracle,
+and against pure fp64 that bound widened by the deviation the rounding of
+dlogits produces (tests/error_model.py), as for the block.
 """
 
 import numpy as np
@@ -13,6 +14,7 @@ import torch
 
 from gemm_epilogue_fusion_tmem_b200 import synth
 from oracle import coda_oracle as O
+from tests import error_model as E
 from tests.parity import assert_pure, assert_tol, f64
 
 pytestmark = pytest.mark.gpu
@@ -35,9 +37,10 @@ def _check(o, b, t, M, d, V, tag):
     if b is not None:
         bs = O.xent_backward(dloss, X, W, tg, fwd=fwd, store=O.round_bf16)
         b0 = O.xent_backward(dloss, X, W, tg, fwd=fwd)
+        sg = E.sigma(E.stored_operand_var(b0["dlogits"], X, W))
         for k in ("dX", "dW"):
             assert_tol(b[k], bs[k], f"{tag} {k}")
-            assert_pure(b[k], b0[k], f"{tag} {k}")
+            assert_pure(b[k], b0[k], f"{tag} {k}", sg[k])
 
 
 @pytest.mark.parametrize("M,d,V", CASES)

@@ -388,6 +388,80 @@ def test_stored_rounding_is_small_and_present():
     assert 1e-4 < rel < 2 ** -8
 
 
+def _placement(case):
+    with open(os.path.join(GOLDEN, "storage_placement.json")) as f:
+        c = json.load(f)["cases"][case]
+    inp = {k: (np.array(v, dtype=np.float64) if isinstance(v, list) else float(v)) for k, v in c["inputs"].items()}
+    return inp, c
+
+
+def _evx(e):
+    return np.array([_evx(x) for x in e]) if isinstance(e, list) else \
+        eval(e, {"exp": math.exp, "sqrt": math.sqrt, "__builtins__": {}})
+
+
+def test_storage_placement_H_rounded_before_r():
+    """H on a bf16 midpoint: the stored H (ties to even) feeds r, so r = 1
+    exactly; computing r from the unrounded H, or rounding ties away from
+    zero, gives r < 1 (tests/golden/storage_placement.json, H_midpoint)."""
+    p, c = _placement("H_midpoint")
+    f = O.grg_forward_stored(p["X"], p["W1"], p["R"], p["g"], p["W2"], p["eps"])
+    e = c["expected"]
+    np.testing.assert_array_equal(f["H"][0], _evx(e["H"]))
+    for k in ("r",):
+        assert f[k][0] == _evx(e[k])
+    for k in ("a", "b"):
+        assert f[k][0, 0] == _evx(e[k])
+    assert f["Y"][0, 0] == pytest.approx(_evx(e["Y"]), rel=1e-15)
+    # the textbook oracle keeps the exact H, and its r differs from the stored one
+    f0 = O.grg_forward(p["X"], p["W1"], p["R"], p["g"], p["W2"], p["eps"])
+    assert f0["r"][0] == pytest.approx(_evx(c["textbook"]["r"]), rel=1e-15)
+    assert f0["r"][0] < f["r"][0]
+
+
+def test_storage_placement_Y_from_unrounded_pre_activations():
+    """a = 1 + 2^-8 sits on a bf16 midpoint: Y is computed from the unrounded
+    a, while the saved a_s is rounded (to 1) (a_midpoint)."""
+    p, c = _placement("a_midpoint")
+    f = O.grg_forward_stored(p["X"], p["W1"], p["R"], p["g"], p["W2"], p["eps"])
+    e = c["expected"]
+    assert f["a"][0, 0] == _evx(e["a"])
+    assert f["a_s"][0, 0] == _evx(e["a_s"]) and f["b_s"][0, 0] == _evx(e["b_s"])
+    assert f["Y"][0, 0] == pytest.approx(_evx(e["Y"]), rel=1e-15)
+    assert abs(f["Y"][0, 0] - float(O.silu(1.0))) > 1e-3
+
+
+def test_storage_placement_gemm2_adjoint_reads_r_scaled_gradient():
+    """r = 1/3: the backward rounds dZ = r [da, db] (171/512), not [da, db]
+    (which is exact at 1), and every weight and input gradient follows from
+    that operand (dZ_row_scale_third)."""
+    p, c = _placement("dZ_row_scale_third")
+    f = O.grg_forward_stored(p["X"], p["W1"], p["R"], p["g"], p["W2"], p["eps"])
+    b = O.grg_backward_stored(p["dY"], p["X"], p["W1"], p["R"], p["g"], p["W2"], p["eps"], fwd=f)
+    e = c["expected"]
+    np.testing.assert_array_equal(b["dZ"][0], _evx(e["dZ"]))
+    np.testing.assert_array_equal(b["dW2"], _evx(e["dW2"]))
+    np.testing.assert_array_equal(b["dg"], _evx(e["dg"]))
+    np.testing.assert_array_equal(b["dR"][0], _evx(e["dR"]))
+    np.testing.assert_array_equal(b["dX"][0], _evx(e["dX"]))
+    np.testing.assert_array_equal(b["dW1"], _evx(e["dW1"]))
+    b0 = O.grg_backward(p["dY"], p["X"], p["W1"], p["R"], p["g"], p["W2"], p["eps"])
+    np.testing.assert_allclose(b0["dR"][0], [1 / 3, -1 / 3], rtol=1e-15)
+    np.testing.assert_allclose(b0["dW2"], [[1, 1], [0, 0]], rtol=1e-15, atol=1e-300)
+
+
+def test_storage_placement_activation_gain_from_stored_H():
+    """With the gain on the activation side, Hg = bf16(stored H * g) = 1.5, not
+    bf16(exact H * g) = 1.5078125; the folded-weight placement gives the same
+    a, b, Y here (activation_gain_from_stored_H)."""
+    p, c = _placement("activation_gain_from_stored_H")
+    e = c["expected"]
+    for gain in ("activation", "weight"):
+        f = O.grg_forward_stored(p["X"], p["W1"], p["R"], p["g"], p["W2"], p["eps"], gain=gain)
+        assert f["a"][0, 0] == _evx(e["a"]) and f["b"][0, 0] == _evx(e["b"]), gain
+        assert f["Y"][0, 0] == pytest.approx(_evx(e["Y"]), rel=1e-15)
+
+
 # ----------------------------------------------------------------------------- cross-entropy
 
 def test_xent_uniform_logits_closed_form():
