@@ -3,7 +3,8 @@
 
 One step = one pass of the whole hot path over one batch of synthetic
 LLaMA-shaped input: for the GRG workloads the gain fold, GEMM1 + residual +
-partial RMS, the row reduce, GEMM2 + r + SwiGLU, and (fwd+bwd workloads) the
+partial RMS, GEMM2 + r (reduced from the partials in its epilogue) + SwiGLU,
+and (fwd+bwd workloads) the
 SwiGLU backward + row statistic, the dn GEMM, the dg column reduce, the dW2,
 dX and dW1 GEMMs.  All of it runs in libcoda.so through the C ABI.
 
@@ -31,6 +32,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "fused GEMM-RMSNorm-GEMM fwd+bwd TFLOP/s and % of B200 bf16 tensor peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+DENSE_BF16_FLOP_PER_SM_CLK = 8192  # tcgen05 dense bf16: 4096 multiply-adds per SM per clock
 
 WORKLOADS = {
     "tiny": ("grg", dict(M=256, K=512, d=512, F=1024, eps=1e-6), True),
@@ -54,6 +56,10 @@ def _args():
     p.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed oracle sample")
     p.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
     p.add_argument("--no-unfused", action="store_true", help="skip timing the unfused comparison sequence")
+    p.add_argument("--no-extra", action="store_true", help="skip timing the 70B shape beside the 7B headline")
+    p.add_argument("--only", choices=["fused", "activation_gain", "unfused"], default=None,
+                   help="profiling aid: run the warm-up steps and then exactly one step of this path, "
+                        "print its kernel launches per step and exit (no timing, no JSON contract line)")
     return p.parse_args()
 
 
@@ -197,7 +203,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={CLOCK_FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             time.sleep(0.3)
         except OSError:
             self.proc = None
@@ -354,7 +360,7 @@ def _make_step(kind, s, bwd, dev):
         step.fwd, step.bwd = fwd_only, (bwd_only if bwd else None)
         outs = {**fo, **bo}
         keys = ["Y", "dX", "dR", "dW1", "dW2", "dg"] if bwd else ["Y", "H", "r"]
-        return step, outs, (10 if bwd else 4), keys, ws
+        return step, outs, (9 if bwd else 3), keys, ws
     if kind == "block":
         K, d, F = s["K"], s["d"], s["F"]
         ws = B.Workspace(max(lib.coda_mlp_block_fwd_workspace_bytes(M, K, d, F),
@@ -368,7 +374,7 @@ def _make_step(kind, s, bwd, dev):
             B.mlp_block_bwd(dev["dOut"], dev["X"], dev["W1"], fo["H"], fo["r"], fo["AB"], fo["Y"], dev["g"],
                             dev["W2"], dev["Wdown"], out=bo, ws=ws)
 
-        return bstep, {**fo, **bo}, 13, ["Out", "dX", "dR", "dW1", "dW2", "dg", "dWdown"], ws
+        return bstep, {**fo, **bo}, 12, ["Out", "dX", "dR", "dW1", "dW2", "dg", "dWdown"], ws
     if kind == "rope":
         a = (s["n_q"], s["n_kv"], s["head_dim"], s["seq_len"], s["base"])
         ws = B.Workspace(lib.coda_qkv_rope_bwd_workspace_bytes(M, s["d"], s["n_q"], s["n_kv"], s["head_dim"]),
@@ -494,17 +500,141 @@ def _time_interleaved(fa, fb, steps, warmup, device, world, barrier, rounds=6):
     return statistics.median(ta), statistics.median(tb)
 
 
+def _make_hg_step(s, bwd, dev, outs, device):
+    """The GRG step with the gain on the activation side (coda_grg_fwd_hg: GEMM1's
+    epilogue stores Hg = bf16(H g), GEMM2 reads the unfolded W2), writing into
+    the same output buffers as the folded-gain step."""
+    from gemm_epilogue_fusion_tmem_b200 import binding as B
+    lib = B.library()
+    hws = B.Workspace(max(lib.coda_grg_fwd_hg_workspace_bytes(s["M"], s["K"], s["d"], 2 * s["F"], 0),
+                          lib.coda_grg_bwd_workspace_bytes(s["M"], s["K"], s["d"], 2 * s["F"])), device)
+    hf = {k: outs[k] for k in ("H", "r", "Y", "AB")}
+    hb = {k: outs[k] for k in ("dX", "dR", "dW1", "dW2", "dg")} if bwd else {}
+
+    def hstep():
+        B.grg_fwd_hg(dev["X"], dev["W1"], dev["R"], dev["g"], dev["W2"], s["eps"], out=hf, ws=hws)
+        if bwd:
+            B.grg_bwd(dev["dY"], dev["X"], dev["W1"], hf["H"], hf["r"], hf["AB"], dev["g"], dev["W2"], out=hb,
+                      ws=hws)
+
+    return hstep, hws
+
+
+def _in_step_kernel_ms(step, epi, steps):
+    """Mean duration of the first launch with epilogue `epi` in each of `steps`
+    back-to-back steps (the library's event hook on the launching stream)."""
+    import torch
+    from gemm_epilogue_fusion_tmem_b200 import binding as B
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    torch.cuda.synchronize()
+    for x, y in ev:
+        B.profile_arm(epi, x, y)
+        step()
+    torch.cuda.synchronize()
+    B.profile_arm(epi)
+    return sum(x.elapsed_time(y) for x, y in ev) / steps
+
+
+def grg_extra(name, a, device, world, barrier):
+    """Another GRG workload timed in the same run (the 70B shape beside the 7B
+    headline): the step with the folded gain, with the gain on the activation
+    side, and the unfused sequence, in alternating bursts (medians), plus the
+    gate/up GEMM's in-step launch time against the burst peak."""
+    import torch
+    kind, s, bwd = WORKLOADS[name]
+    host, dev = _setup(kind, s, bwd, device)
+    del host
+    step, outs, launches, _, ws = _make_step(kind, s, bwd, dev)
+    hstep, hws = _make_hg_step(s, bwd, dev, outs, device)
+    ustep, ulaunch, uws = _make_unfused_step(kind, s, bwd, dev)
+    flops = _flops(kind, s, bwd)
+    f_ms, u_ms = _time_interleaved(step, ustep, a.steps, a.warmup, device, world, barrier)
+    h_ms, u2_ms = _time_interleaved(hstep, ustep, a.steps, a.warmup, device, world, barrier)
+    fd, ud = _time_interleaved(step.fwd, ustep.fwd, a.steps, a.warmup, device, world, barrier)
+    peaks, src = _peaks()
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    k_flops = 2.0 * s["M"] * s["d"] * 2 * s["F"]
+    kh = _in_step_kernel_ms(hstep, DOMINANT_EPI[kind], max(a.steps, 5))
+    kf = _in_step_kernel_ms(step, DOMINANT_EPI[kind], max(a.steps, 5))
+    status, detail = ws.query()
+    if status != 0:
+        raise SystemExit(f"bench.py: device status {status} detail {detail:#x} in the {name} extra")
+    rate = lambda ms: round(replica_throughput(flops, 1, world, ms), 2)  # noqa: E731
+    out = {"config": _describe(name, kind, s, bwd), "flops_per_step": flops,
+           "timing": "alternating bursts (fused, unfused, fused, ...), median ms per step of each",
+           "fused_folded_gain": {"ms_per_step": round(f_ms, 4), "value": rate(f_ms),
+                                 "frac_of_burst": round(rate(f_ms) / world / burst, 4),
+                                 "unfused_ms_per_step": round(u_ms, 4), "speedup_vs_unfused": round(u_ms / f_ms, 4),
+                                 "fwd": {"fused_ms": round(fd, 4), "unfused_ms": round(ud, 4),
+                                         "speedup": round(ud / fd, 4)},
+                                 "gate_up_gemm_in_step_ms": round(kf, 4),
+                                 "gate_up_gemm_frac_of_burst": round(k_flops / (kf / 1e3) / 1e12 / burst, 4)},
+           "fused_activation_gain": {"ms_per_step": round(h_ms, 4), "value": rate(h_ms),
+                                     "frac_of_burst": round(rate(h_ms) / world / burst, 4),
+                                     "unfused_ms_per_step": round(u2_ms, 4),
+                                     "speedup_vs_unfused": round(u2_ms / h_ms, 4),
+                                     "gate_up_gemm_in_step_ms": round(kh, 4),
+                                     "gate_up_gemm_frac_of_burst": round(k_flops / (kh / 1e3) / 1e12 / burst, 4)},
+           "unfused": {"value": rate(u_ms), "gpu_launches_per_step": ulaunch},
+           "peak": {"bf16_burst_tflops": burst, "source": src},
+           "unit": "TFLOP/s"}
+    del ws, hws, uws, outs, dev, step, hstep, ustep
+    torch.cuda.empty_cache()
+    return out
+
+
+def epilogue_ab(kind, s, dev, outs, a, device, world, barrier):
+    """The dominant gate/up GEMM with its r + SwiGLU epilogue against a plain
+    store of the same [M, 2F] product (same operands, same kernel, epilogue
+    swapped), in alternating bursts with the SM clock sampled in each: the
+    epilogue's cost at equal clocks is time x MHz."""
+    import torch
+    from gemm_epilogue_fusion_tmem_b200 import binding as B
+    if kind not in ("grg", "block", "swiglu"):
+        return None
+    if kind in ("grg", "block"):
+        A, W, r = outs["H"], dev["W2"], outs["r"]
+    else:
+        A, W, r = dev["X"], dev["Wgu"], None
+    M, K, F = s["M"], s["d"], s["F"]
+    o = {"Y": torch.empty(M, F, dtype=torch.bfloat16, device=device),
+         "AB": torch.empty(M, 2 * F, dtype=torch.bfloat16, device=device)}
+    C = torch.empty(M, 2 * F, dtype=torch.bfloat16, device=device)
+    fused = lambda: B.gemm_swiglu(A, W, r, out=o)  # noqa: E731
+    plain = lambda: B.gemm(A, W, M, 2 * F, K, out=C)  # noqa: E731
+    for _ in range(3):
+        fused()
+        plain()
+    # Bursts of about 250 ms, long enough for several 50 ms clock samples.
+    per = max(10, int(250.0 / max(_time_loop(fused, 3, None, device, world, barrier) / 3, 1e-3)))
+    tf, tp, cf, cp = [], [], [], []
+    for _ in range(4):
+        with ClockSampler(device.index) as c1:
+            tf.append(_time_loop(fused, per, None, device, world, barrier) / per)
+        with ClockSampler(device.index) as c2:
+            tp.append(_time_loop(plain, per, None, device, world, barrier) / per)
+        cf.append(c1.summary().get("sm_mhz"))
+        cp.append(c2.summary().get("sm_mhz"))
+    med = statistics.median
+    mf, mp = med(tf), med(tp)
+    out = {"swiglu_ms": round(mf, 4), "plain_store_ms": round(mp, 4), "ratio": round(mf / mp, 4),
+           "timing": f"4 alternating bursts of {per} launches each, medians"}
+    cf, cp = [x for x in cf if x], [x for x in cp if x]
+    if cf and cp:
+        out["sm_mhz"] = {"swiglu": med(cf), "plain_store": med(cp)}
+        out["ratio_at_equal_clock"] = round(mf * med(cf) / (mp * med(cp)), 4)
+    return out
+
+
 def _grg_kernels(s, bwd):
     """The block's kernels in launch order with their algorithmic work per launch:
     (hook id, name, bound, amount) with FLOPs for tensor-bound GEMMs and
     compulsory HBM bytes for the light passes."""
     M, K, d, F = s["M"], s["K"], s["d"], s["F"]
     N = 2 * F
-    T = -(-d // 256)  # partial sums per row (one per 256-column tile)
     ks = [(16, "fold_gain (W2g = W2 diag g)", "hbm", 4.0 * N * d + 2.0 * d),
           (1, "GEMM1 + residual + partial sums", "tensor", 2.0 * M * K * d),
-          (17, "row reduce -> r", "hbm", 4.0 * M * T + 4.0 * M),
-          (2, "GEMM2 + r + SwiGLU", "tensor", 2.0 * M * d * N)]
+          (2, "GEMM2 + r (from the partial sums) + SwiGLU", "tensor", 2.0 * M * d * N)]
     if bwd:
         rows = -(-M // 256) * 256 // 32  # dg partial rows: one per 32 output rows
         ks += [(18, "SwiGLU bwd + row coefficient", "hbm", 2.0 * M * F + 4.0 * M * N + 8.0 * M),
@@ -738,22 +868,41 @@ def run_coda(a):
     ms_max = max_over_ranks(ms_total, device, world)
     value = replica_throughput(flops, a.steps, world, ms_max)
 
+    # The same step once the power cap has settled: about two seconds of
+    # back-to-back steps, then the same number of steps timed again (the
+    # headline region above starts right after the warm-up, a short burst).
+    n_pre = max(1, int(2000.0 / max(ms_total / a.steps, 1e-3)))
+    n_set = max(a.steps, int(1000.0 / max(ms_total / a.steps, 1e-3)))  # at least a second, for clock samples
+    kev_s = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_set)]
+    with ClockSampler(local) as clk_settled:
+        for _ in range(n_pre):
+            step()
+        torch.cuda.synchronize()
+        barrier()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(st)
+        for i in range(n_set):
+            B.profile_arm(k_epi, *kev_s[i])
+            step()
+        s1.record(st)
+        torch.cuda.synchronize()
+        barrier()
+    B.profile_arm(k_epi)
+    settled_ms = max_over_ranks(s0.elapsed_time(s1), device, world)
+    k_set_ms = sum(x.elapsed_time(y) for x, y in kev_s) / n_set
+    settled = {"ms_per_step": round(settled_ms / n_set, 4),
+               "value": round(replica_throughput(flops, n_set, world, settled_ms), 2), "steps": n_set,
+               "after_steps": n_pre, "clocks": clk_settled.summary(),
+               "dominant_kernel_ms": round(k_set_ms, 4),
+               "how": f"{n_pre} untimed back-to-back steps (about 2 s), then {n_set} steps (about 1 s) timed "
+                      f"like the headline"}
+
     # The activation-side gain variant (Hg from GEMM1's epilogue, no gain fold).
     variants = {}
     if kind == "grg":
         from gemm_epilogue_fusion_tmem_b200 import binding as B
         lib = B.library()
-        hws = B.Workspace(max(lib.coda_grg_fwd_hg_workspace_bytes(s["M"], s["K"], s["d"], 2 * s["F"], 0),
-                              lib.coda_grg_bwd_workspace_bytes(s["M"], s["K"], s["d"], 2 * s["F"])), device)
-        hf = {k: outs[k] for k in ("H", "r", "Y", "AB")}
-        hb = {k: outs[k] for k in ("dX", "dR", "dW1", "dW2", "dg")} if bwd else {}
-
-        def hstep():
-            B.grg_fwd_hg(dev["X"], dev["W1"], dev["R"], dev["g"], dev["W2"], s["eps"], out=hf, ws=hws)
-            if bwd:
-                B.grg_bwd(dev["dY"], dev["X"], dev["W1"], hf["H"], hf["r"], hf["AB"], dev["g"], dev["W2"], out=hb,
-                          ws=hws)
-
+        hstep, hws = _make_hg_step(s, bwd, dev, outs, device)
         f_ms, h_ms = _time_interleaved(step, hstep, a.steps, a.warmup, device, world, barrier)
         variants["activation_gain"] = {"ms_per_step": round(h_ms, 4),
                                        "value": round(replica_throughput(flops, 1, world, h_ms), 2),
@@ -807,21 +956,50 @@ def run_coda(a):
         del uws
 
     # Roofline of the dominant kernel: its average launch duration inside the
-    # timed steps (a kernel inside a long, power-limited step: the sustained
-    # peak), with the same kernel timed alone against the burst peak beside it.
+    # timed steps.  The timed region is a short burst unless it runs for more
+    # than a second, so the burst peak is the denominator then (the sustained
+    # one, a seconds-long loop under the power cap, otherwise).  Beside it the
+    # same kernel timed alone, and the fraction of the dense bf16 rate at the
+    # SM clock measured under load in the timed region.
     peaks, peaks_src = _peaks()
     achieved = k_flops / (k_ms / 1e3) / 1e12
-    peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    long_region = ms_total > 1000.0
+    peak = sustained if long_region else burst
     alone = k_flops / (k_alone_ms / 1e3) / 1e12
+    clk_head = clk.summary()
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    # The headline region (about 0.1 s at the driver's 20 steps) holds too few
+    # 50 ms clock samples under load to know its clock; the settled region
+    # (a second or more) does, so the clock-normalised fraction is taken there.
+    clk_set = settled["clocks"]
+    set_mhz = clk_set.get("sm_mhz") if clk_set.get("samples_under_load", 0) >= 5 else None
+    at_clock = (sms * DENSE_BF16_FLOP_PER_SM_CLK * set_mhz * 1e6 / 1e12) if set_mhz else None
+    achieved_set = k_flops / (settled["dominant_kernel_ms"] / 1e3) / 1e12
     roofline = {"bound": "tensor", "kernel": kname, "achieved": round(achieved, 1), "peak": peak,
                 "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                 "traffic": _recorded_traffic(kname, a.workload),
-                "peak_source": f"{peaks_src} sustained bf16 (kernel timed inside the timed steps)",
+                "peak_source": (f"{peaks_src} {'sustained' if long_region else 'burst'} bf16 "
+                                f"(timed region {ms_total:.0f} ms: "
+                                f"{'longer' if long_region else 'shorter'} than 1 s)"),
                 "launch_ms": round(k_ms, 4), "launches_timed": a.steps,
+                "flops_per_launch": k_flops,
+                "clock_normalised": None if at_clock is None else {
+                    "region": "settled", "launch_ms": settled["dominant_kernel_ms"],
+                    "achieved": round(achieved_set, 1), "sm_mhz": set_mhz, "sms": sms,
+                    "dense_bf16_at_clock": round(at_clock, 1), "frac": round(achieved_set / at_clock, 4),
+                    "how": f"the kernel's mean launch time in the settled steps against {sms} SMs x "
+                           f"{DENSE_BF16_FLOP_PER_SM_CLK} dense bf16 FLOP per SM clock x the median SM clock "
+                           f"sampled under load there"},
                 "alone": {"launch_ms": round(k_alone_ms, 4), "achieved": round(alone, 1), "peak": burst,
                           "frac": round(alone / burst, 4),
                           "peak_source": f"{peaks_src} burst bf16 (kernel timed alone, after warm-up)"}}
+
+    # The dominant kernel's epilogue against a plain store of the same product.
+    epi_ab = epilogue_ab(kind, s, dev, outs, a, device, world, barrier)
+    if epi_ab is not None:
+        roofline["epilogue_vs_plain_store"] = epi_ab
 
     # Every kernel of the step timed on its own (light passes in GB/s against HBM).
     breakdown = _kernel_breakdown(kind, s, bwd, step)
@@ -835,12 +1013,17 @@ def run_coda(a):
     if not a.no_e2e:
         e2e = _e2e_pipelined(kind, s, bwd, host, dev, step, outs, result_keys, flops, a, device, world, barrier)
 
+    # The 70B shape timed in the same run beside the 7B headline.
+    extra = {}
+    if a.workload == "7B" and not a.no_extra:
+        extra["70B"] = grg_extra("70B", a, device, world, barrier)
+
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         cpu = cpu_baseline(kind, s, bwd)
 
     if rank == 0:
-        frac_step = value / world / float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+        per_gpu = value / world
         line = {
             "metric": METRIC,
             "value": round(value, 2),
@@ -857,15 +1040,20 @@ def run_coda(a):
             "config": {**_describe(a.workload, kind, s, bwd), "parallelism": f"replicas x{world}",
                        "l2": l2_note,
                        "l2_flushed": l2_flushed,
-                       "flops_per_step": flops, "frac_of_sustained_bf16_peak": round(frac_step, 4)},
+                       "flops_per_step": flops, "timed_region_ms": round(ms_max, 2),
+                       "frac_of_bf16_peak": {"burst": round(per_gpu / burst, 4),
+                                             "sustained": round(per_gpu / sustained, 4),
+                                             "source": peaks_src}},
             "roofline": roofline,
+            "settled": settled,
             "kernels": breakdown,
+            "extra": extra or None,
             "cpu_baseline": cpu,
             "unfused": unfused,
             "variants": variants or None,
             "e2e": e2e,
             "gpu_launches": launches * a.steps,
-            "clocks": clk.summary(),
+            "clocks": clk_head,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -911,10 +1099,39 @@ def run_reference(a):
     return line
 
 
+def run_only(a):
+    """One step of one path after the warm-up steps, for a profiler's launch list:
+    the captured launches are those after warmup x launches-per-step."""
+    import torch
+    kind, s, bwd = WORKLOADS[a.workload]
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    host, dev = _setup(kind, s, bwd, device)
+    del host
+    if a.only == "unfused":
+        step, launches, ws = _make_unfused_step(kind, s, bwd, dev)
+    else:
+        step, outs, launches, _, ws = _make_step(kind, s, bwd, dev)
+        if a.only == "activation_gain":
+            step, ws = _make_hg_step(s, bwd, dev, outs, device)
+            launches -= 1  # no gain fold
+    for _ in range(a.warmup):
+        step()
+    step()
+    torch.cuda.synchronize()
+    status, detail = ws.query()
+    if status != 0:
+        raise SystemExit(f"bench.py --only: device status {status} detail {detail:#x}")
+    print(json.dumps({"only": a.only, "workload": a.workload, "warmup": a.warmup,
+                      "launches_per_step": launches}), flush=True)
+
+
 def main():
     a = _args()
     if a.impl == "reference":
         run_reference(a)
+    elif a.only is not None:
+        run_only(a)
     else:
         run_coda(a)
 

@@ -151,7 +151,6 @@ template <typename Fn>
 int aux_tag(Fn kern) {
   const void* f = reinterpret_cast<const void*>(kern);
   if (f == reinterpret_cast<const void*>(fold_gain_kernel)) return CODA_KERNEL_FOLD_GAIN;
-  if (f == reinterpret_cast<const void*>(rms_rowreduce_kernel)) return CODA_KERNEL_RMS_ROWREDUCE;
   if (f == reinterpret_cast<const void*>(swiglu_bwd_rowstat_kernel)) return CODA_KERNEL_SWIGLU_BWD_ROWSTAT;
   if (f == reinterpret_cast<const void*>(col_reduce_kernel)) return CODA_KERNEL_COL_REDUCE;
   if (f == reinterpret_cast<const void*>(rowcoef_reduce_kernel)) return CODA_KERNEL_ROWCOEF_REDUCE;
@@ -212,6 +211,17 @@ int raster_budget_mb() {
   }();
   return v;
 }
+// Distance, in k-blocks, at which the TMA producer prefetches operand boxes
+// into L2 ahead of its loads (CODA_L2_PREFETCH; 0 turns prefetching off).
+int l2_prefetch_stages() {
+  static const int v = [] {
+    const char* e = std::getenv("CODA_L2_PREFETCH");
+    const int x = e ? std::atoi(e) : 0;
+    return x > 0 ? std::min(x, 64) : 0;
+  }();
+  return v;
+}
+
 int pick_group(long long a_rows, long long b_rows, long long K, int num_m, int num_n, bool pair, int num_sms) {
   const int units = pair ? num_sms / 2 : num_sms;
   int side = 1;
@@ -273,6 +283,7 @@ coda_status launch_gemm_mode(const CUtensorMap& ta, const CUtensorMap& tb, GemmP
     return CODA_ERR_CUDA;
   p.kernel_id = (uint32_t)(slot + 1);
   p.wait_limit_ns = g_wait_limit_ns.load();
+  p.prefetch_stages = l2_prefetch_stages();
   if (p.group_m == 0) p.group_m = 1;
   const int tiles = p.num_m_tiles * p.num_n_tiles;
   const int units = std::min(tiles, di.max_clusters[slot]);  // persistent: one tile stream per CTA (pair)
@@ -328,9 +339,20 @@ coda_status gemm_store(const void* A, const void* B, void* C, int M, int N, int 
 
 coda_status launch_status(cudaError_t e) { return e == cudaSuccess ? CODA_OK : CODA_ERR_CUDA; }
 
-// Gate/up GEMM with the row-scale + SwiGLU epilogue (r may be null).
+// The RMSNorm row scale's source for the gate/up GEMM: the partial sums of
+// squares P [M, T] of GEMM1's epilogue, from which the epilogue forms r and
+// stores it to r_out (the block's forward, no separate row reduce).
+struct RowScaleFromPartials {
+  const float* P;
+  int T;
+  float inv_d, eps;
+  float* r_out;
+};
+
+// Gate/up GEMM with the row-scale + SwiGLU epilogue: r from `rs` when given,
+// else read from r (which may be null: no row scale).
 coda_status gemm_swiglu(const void* A, const void* Wgu, const float* r, void* Y, void* AB, int M, int K, int F,
-                        void* ws, cudaStream_t s) {
+                        void* ws, cudaStream_t s, const RowScaleFromPartials* rs = nullptr) {
   CUtensorMap ta, tb;
   if (!make_operand_map(&ta, A, M, K, false, BM) || !make_operand_map(&tb, Wgu, 2LL * F, K, false, BN / 2))
     return CODA_ERR_CUDA;
@@ -343,6 +365,13 @@ coda_status gemm_swiglu(const void* A, const void* Wgu, const float* r, void* Y,
   p.out2 = bf(AB);
   p.ldo2 = 2 * F;
   p.rowvec = r;
+  if (rs != nullptr) {
+    p.part = const_cast<float*>(rs->P);
+    p.ld_part = rs->T;
+    p.inv_d = rs->inv_d;
+    p.eps = rs->eps;
+    p.outf = rs->r_out;
+  }
   return launch_gemm<EPI_SWIGLU, false, false>(ta, tb, p, s, pair);
 }
 
@@ -571,12 +600,10 @@ coda_status coda_grg_fwd(const void* X, const void* W1, const void* R, const voi
     p.ld_part = T;
     CODA_TRY((launch_gemm<EPI_RESID_RMS, false, false>(ta, tb, p, s, pair)));
   }
-  // Row reduce -> r.
-  CODA_TRY(launch_status(launch_ex(rms_rowreduce_kernel, dim3(cdiv(M, 256)), dim3(256), 0, s, 1, (const float*)P, T,
-                                   r, M, 1.0f / (float)d, eps)));
-  // GEMM2 (gate|up) + r scaling + SwiGLU.
-  CODA_TRY(gemm_swiglu(H, W2g, r, Y, AB_or_null, M, d, F, ws, s));
-  return CODA_OK;
+  // GEMM2 (gate|up): its epilogue forms r from the partial sums (the light
+  // row reduction), stores it, scales the rows by it and applies SwiGLU.
+  const RowScaleFromPartials rs{P, T, 1.0f / (float)d, eps, r};
+  return gemm_swiglu(H, W2g, nullptr, Y, AB_or_null, M, d, F, ws, s, &rs);
 }
 
 size_t coda_grg_fwd_hg_workspace_bytes(int M, int K, int d, int N, int hg_given) {
@@ -624,9 +651,8 @@ coda_status coda_grg_fwd_hg(const void* X, const void* W1, const void* R, const 
     p.colvec = cbf(g);
     CODA_TRY((launch_gemm<EPI_RESID_RMS, false, false>(ta, tb, p, s, pair)));
   }
-  CODA_TRY(launch_status(launch_ex(rms_rowreduce_kernel, dim3(cdiv(M, 256)), dim3(256), 0, s, 1, (const float*)P, T,
-                                   r, M, 1.0f / (float)d, eps)));
-  return gemm_swiglu(Hg, W2, r, Y, AB_or_null, M, d, F, ws, s);
+  const RowScaleFromPartials rs{P, T, 1.0f / (float)d, eps, r};
+  return gemm_swiglu(Hg, W2, nullptr, Y, AB_or_null, M, d, F, ws, s, &rs);
 }
 
 // ------------------------------------------------------------------ GRG backward
@@ -1290,9 +1316,8 @@ extern "C" coda_status coda_grg_fwd_prefolded_static(const void* X, const void* 
     p.ld_part = T;
     CODA_TRY((launch_gemm<EPI_RESID_RMS, false, false>(ta, tb, p, s, pair)));
   }
-  CODA_TRY(launch_status(launch_ex(rms_rowreduce_kernel, dim3(cdiv(M, 256)), dim3(256), 0, s, 1, (const float*)P, T,
-                                   r, M, 1.0f / (float)d, eps)));
-  return gemm_swiglu(H, W2g, r, Y, AB_or_null, M, d, F, scratch, s);
+  const RowScaleFromPartials rs{P, T, 1.0f / (float)d, eps, r};
+  return gemm_swiglu(H, W2g, nullptr, Y, AB_or_null, M, d, F, scratch, s, &rs);
 }
 
 extern "C" coda_status coda_static_status_query(void* stream, uint32_t* detail) {

@@ -1,6 +1,9 @@
-// The light HBM-bound passes around the GEMMs: gain fold, row reduce of the
-// partial sums of squares, SwiGLU backward with its row statistic, and the
-// column reduce of the dg partials.  All use 16-byte vector accesses.
+// The light HBM-bound passes around the GEMMs: gain fold, SwiGLU backward
+// with its row statistic, and the column reduce of the dg partials.  All use
+// 16-byte vector accesses.  (The row reduce of the partial sums of squares,
+// the "very light auxiliary reduction" of the kucoin.com (ru) CODA article,
+// section «В «Финале» спрятаны сокровища», runs in the gate/up GEMM's
+// epilogue, see swiglu_row_scale in coda_gemm.cuh.)
 #pragma once
 
 #include "coda_ptx.cuh"
@@ -44,20 +47,6 @@ __global__ void fold_gain_kernel(const __nv_bfloat16* __restrict__ W2, const __n
       stg_v4(W2g + vu * 8, pack8(f));
     }
   }
-}
-
-// r_i = 1 / sqrt(sum_t P[i, t] / d + eps): the "very light auxiliary
-// reduction" that turns GEMM1's partial RMS into the RMSNorm row scale
-// (kucoin.com (ru) CODA article, «В «Финале» спрятаны сокровища»).
-__global__ void rms_rowreduce_kernel(const float* __restrict__ P, int T, float* __restrict__ r, int M,
-                                     float inv_d, float eps) {
-  griddep_wait();
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= M) return;
-  const float* row = P + (size_t)i * T;
-  float s = 0.f;
-  for (int t = 0; t < T; ++t) s += row[t];
-  r[i] = rsqrtf(fmaf(s, inv_d, eps));
 }
 
 // c_i = (r_i^2 / d) sum_t Pc[i, t]: the RMSNorm backward's row coefficient

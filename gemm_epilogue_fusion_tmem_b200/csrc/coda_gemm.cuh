@@ -68,17 +68,20 @@ struct GemmParams {
   const __nv_bfloat16* in1;  // dH_in (DN), optional
   const __nv_bfloat16* colvec;  // g (STORE scale, DN), optional for STORE
   const float* rowvec;          // r (SWIGLU, optional), c (DN)
-  float* part;                  // P (RESID_RMS), Pg (DN)
+  float* part;                  // P (RESID_RMS; read by SWIGLU to form r), Pg (DN)
   int ld_part;
   __nv_bfloat16* out2;          // AB (SWIGLU), Hg (RESID_RMS), optional
   int ldo2;
   const int* tgt;               // target class per row (XENT, XENT_BWD)
   const float* rowvec2;         // dloss (XENT_BWD)
-  float* outf;                  // target logit per row (XENT)
+  float* outf;                  // target logit per row (XENT); r (SWIGLU with part)
   int head_dim;                 // ROPE: head width (64, 128 or 256)
   int rot_cols;                 // ROPE: columns [0, rot_cols) are rotated (q and k heads)
   int seq_len;                  // ROPE: position = row % seq_len
   float rope_k;                 // ROPE: -2 log2(base) / head_dim, so inv_freq_j = 2^(j * rope_k)
+  int prefetch_stages;          // L2 prefetch distance of the producer in stages (0: none)
+  float inv_d;                  // SWIGLU with part: 1 / d of the RMSNorm mean
+  float eps;                    // SWIGLU with part: the RMSNorm eps
   uint32_t* status;
   unsigned long long wait_limit_ns;
   uint32_t kernel_id;
@@ -145,8 +148,12 @@ __device__ __forceinline__ void pref_unpack(const Pref32& x, float (&f)[32]) {
 // bank-conflict free and matches the tensor map's 64-byte swizzle); one lane
 // then issues a TMA bulk tensor store.  TMA clips rows and columns outside
 // the tensor, so ragged row tiles need no masking.  Up to kEpiTiles tiles per
-// 32-column step; the staging is reused once the previous step's stores have
-// been read.
+// 32-column step.  A step that stages one tile rotates over the kEpiTiles
+// slots, so it waits only for the store issued kEpiTiles steps earlier; a step
+// that stages more waits until the previous step's stores have been read.
+// Each output tile starts with all slots free (begin_tile), so a warp whose
+// rows lie past M in one tile (it stages but stores nothing) cannot overwrite
+// a slot that an earlier tile's store is still reading.
 constexpr int kEpiTiles = 3;
 constexpr int kEpiTileBytes = 32 * 32 * 2;
 constexpr int kEpiWarpBytes = kEpiTiles * kEpiTileBytes;
@@ -157,16 +164,32 @@ struct EpiStore {
   int row0;       // first output row of this warp
   int rows;       // output rows (M); a warp wholly past them stores nothing
   int n;          // tiles staged in the current step
+  int base;       // first slot of the current step
+  int slot;       // next slot of a one-tile step
   const CUtensorMap* map[kEpiTiles];
   int col[kEpiTiles];
 
-  __device__ __forceinline__ void begin() {
+  __device__ __forceinline__ void begin_tile() {
     if (lane == 0) bulk_wait_read_all();
+    __syncwarp();
+    slot = 0;
+  }
+  // Reserve the slots of one step that stages `tiles` output tiles.
+  __device__ __forceinline__ void begin(int tiles = kEpiTiles) {
+    static_assert(kEpiTiles == 3, "the rotating wait below allows kEpiTiles - 1 = 2 groups in flight");
+    if (tiles == 1) {
+      if (lane == 0) bulk_wait_read_2();
+      base = slot;
+      slot = (slot + 1 == kEpiTiles) ? 0 : slot + 1;
+    } else {
+      if (lane == 0) bulk_wait_read_all();
+      base = 0;
+    }
     __syncwarp();
     n = 0;
   }
   __device__ __forceinline__ void put_packed(const uint4 (&q)[4], const CUtensorMap* m, int c) {
-    uint8_t* t = stg + n * kEpiTileBytes + lane * 64;
+    uint8_t* t = stg + (base + n) * kEpiTileBytes + lane * 64;
     const int sw = (lane >> 1) & 3;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -189,7 +212,7 @@ struct EpiStore {
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0 && row0 < rows) {
-      for (int t = 0; t < n; ++t) tma_store_2d(map[t], stg + t * kEpiTileBytes, col[t], row0);
+      for (int t = 0; t < n; ++t) tma_store_2d(map[t], stg + (base + t) * kEpiTileBytes, col[t], row0);
       bulk_commit_group();
     }
   }
@@ -216,12 +239,29 @@ __device__ __forceinline__ void warp_column_sums(float (&v)[32], int lane) {
 }
 
 
-// Loads the first chunk of a tile's per-row epilogue inputs (issued before the
-// wait for the accumulator).
+// The RMSNorm row scale for the gate/up GEMM: with GEMM1's partial sums of
+// squares (p.part) it is formed here, r_i = 1/sqrt(sum_t P[i,t] / d + eps),
+// the partials summed in column-tile order, and the row's first column tile
+// stores it; otherwise it is read from p.rowvec (1 when there is none).
+__device__ __forceinline__ float swiglu_row_scale(const GemmParams& p, int row, bool rv, int n_blk) {
+  if (p.part == nullptr) return (p.rowvec != nullptr) ? (rv ? p.rowvec[row] : 0.f) : 1.f;
+  if (!rv) return 0.f;
+  const float* pr = p.part + (size_t)row * p.ld_part;
+  float s = 0.f;
+  for (int t = 0; t < p.ld_part; ++t) s += pr[t];
+  const float r = rsqrtf(fmaf(s, p.inv_d, p.eps));
+  if (n_blk == 0) p.outf[row] = r;
+  return r;
+}
+
+// Loads the first chunk of a tile's per-row epilogue inputs, and the gate/up
+// GEMM's row scale (issued before the wait for the accumulator).
 template <int EPI>
 __device__ __forceinline__ void epilogue_prefetch(const GemmParams& p, int row, bool rv, int n_blk, Pref32& x0,
-                                                  Pref32& x1) {
-  if constexpr (EPI == EPI_RESID_RMS || EPI == EPI_DN) {
+                                                  Pref32& x1, float& rr) {
+  if constexpr (EPI == EPI_SWIGLU) {
+    rr = swiglu_row_scale(p, row, rv, n_blk);
+  } else if constexpr (EPI == EPI_RESID_RMS || EPI == EPI_DN) {
     const size_t off = (size_t)row * p.ld_in0 + (size_t)n_blk * BN;
     pref_load(x0, p.in0 + off, rv);
     if constexpr (EPI == EPI_DN) {
@@ -239,7 +279,7 @@ __device__ __forceinline__ void epilogue_prefetch(const GemmParams& p, int row, 
 template <int EPI>
 __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbase, int row, bool rv, int group32,
                                               int n_blk, int lane, EpiStore& es, const CUtensorMap* mo1,
-                                              const CUtensorMap* mo2, Pref32& x0, Pref32& x1) {
+                                              const CUtensorMap* mo2, Pref32& x0, Pref32& x1, float rr) {
   if constexpr (EPI == EPI_STORE) {
     const int n0 = n_blk * BN;
 #pragma unroll 1
@@ -253,7 +293,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbas
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] *= g[i];
       }
-      es.begin();
+      es.begin(1);
       es.put(v, mo1, n0 + c);
       es.flush();
     }
@@ -279,7 +319,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbas
 #pragma unroll
         for (int i = 0; i < 8; ++i) ss = fmaf(v[8 * j + i], v[8 * j + i], ss);
       }
-      es.begin();
+      es.begin(p.out2 != nullptr ? 2 : 1);
       es.put_packed(hq, mo1, n0 + c);
       if (p.out2 != nullptr) {
         // Activation-side gain: Hg = bf16(H * g) from the stored H, the second
@@ -297,7 +337,6 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbas
   } else if constexpr (EPI == EPI_SWIGLU) {
     constexpr int HALF = BN / 2;
     const int n0 = n_blk * HALF;
-    const float rr = (p.rowvec != nullptr) ? (rv ? p.rowvec[row] : 0.f) : 1.f;
 #pragma unroll 1
     for (int c = 0; c < HALF; c += 32) {
       if (n0 + c >= p.N) break;
@@ -311,7 +350,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbas
         b[i] *= rr;
         y[i] = a[i] * sigmoid_f(a[i]) * b[i];
       }
-      es.begin();
+      es.begin(p.out2 != nullptr ? 3 : 1);
       es.put(y, mo1, n0 + c);
       if (p.out2 != nullptr) {
         es.put(a, mo2, n0 + c);
@@ -343,7 +382,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbas
 #pragma unroll
         for (int i = 0; i < 32; ++i) o[i] += e[i];
       }
-      es.begin();
+      es.begin(1);
       es.put(o, mo1, n0 + c);
       es.flush();
       // dg partial: sum over this warp's 32 rows of acc * H, per column.
@@ -397,7 +436,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbas
         if (i == off) g -= 1.f;
         v[i] = g * dl;
       }
-      es.begin();
+      es.begin(1);
       es.put(v, mo1, n0 + c);
       es.flush();
     }
@@ -488,6 +527,40 @@ struct TileCfg {
   static constexpr int CTAS = PAIR ? 2 : 1;
 };
 
+// L2 prefetch of the operand boxes this CTA loads for k-block kb of `tile`:
+// the same boxes as the producer's loads, issued prefetch_stages stages ahead
+// so that a miss in L2 is served from DRAM while the ring still holds earlier
+// stages.
+template <int EPI, bool A_MN, bool B_MN, bool PAIR>
+__device__ __forceinline__ void prefetch_stage(const CUtensorMap* tmA, const CUtensorMap* tmB, const GemmParams& p,
+                                               int tile, int kb, uint32_t rank) {
+  using C = TileCfg<PAIR>;
+  int m_blk, n_blk;
+  tile_coords(tile, p.num_m_tiles, p.num_n_tiles, p.group_m, m_blk, n_blk);
+  const int a_row = m_blk * C::TILE_M + (int)rank * 128;
+  const int k0 = kb * BK;
+  if constexpr (!A_MN) {
+    tma_prefetch_2d(tmA, k0, a_row);
+  } else {
+#pragma unroll
+    for (int c = 0; c < 2; ++c) tma_prefetch_2d(tmA, a_row + c * 64, k0);
+  }
+  if constexpr (EPI == EPI_SWIGLU) {
+    if constexpr (PAIR) {
+      tma_prefetch_2d(tmB, k0, (rank ? p.split : 0) + n_blk * (BN / 2));
+    } else {
+      tma_prefetch_2d(tmB, k0, n_blk * (BN / 2));
+      tma_prefetch_2d(tmB, k0, p.split + n_blk * (BN / 2));
+    }
+  } else if constexpr (!B_MN) {
+    tma_prefetch_2d(tmB, k0, n_blk * BN + (PAIR ? (int)rank * 128 : 0));
+  } else {
+    constexpr int chunks = PAIR ? 2 : BN / 64;
+#pragma unroll
+    for (int c = 0; c < chunks; ++c) tma_prefetch_2d(tmB, n_blk * BN + (PAIR ? (int)rank * 128 : 0) + c * 64, k0);
+  }
+}
+
 template <int EPI, bool A_MN, bool B_MN, bool PAIR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -563,11 +636,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
+      // L2 prefetch cursor, prefetch_stages k-blocks ahead of the loads.
+      int pf_tile = first_tile, pf_kb = p.prefetch_stages;
+      while (pf_kb >= p.k_blocks && p.prefetch_stages > 0) {
+        pf_kb -= p.k_blocks;
+        pf_tile += tile_step;
+      }
       for (int tile = first_tile; tile < num_tiles && ok; tile += tile_step) {
         int m_blk, n_blk;
         tile_coords(tile, p.num_m_tiles, p.num_n_tiles, p.group_m, m_blk, n_blk);
         const int a_row = m_blk * C::TILE_M + (int)rank * 128;
         for (int kb = 0; kb < p.k_blocks; ++kb) {
+          if (p.prefetch_stages > 0 && pf_tile < num_tiles) {
+            prefetch_stage<EPI, A_MN, B_MN, PAIR>(&tmA, &tmB, p, pf_tile, pf_kb, rank);
+            if (++pf_kb == p.k_blocks) {
+              pf_kb = 0;
+              pf_tile += tile_step;
+            }
+          }
           if (!mbar_wait(&empty[stage], phase ^ 1u, ctl, 0, kWaitEmpty)) {
             ok = false;
             break;
@@ -697,15 +783,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tile_coords(tile, p.num_m_tiles, p.num_n_tiles, p.group_m, m_blk, n_blk);
       const int row0 = m_blk * C::TILE_M + (int)rank * 128 + q * 32;
       Pref32 x0, x1;
-      epilogue_prefetch<EPI>(p, row0 + lane, row0 + lane < p.M, n_blk, x0, x1);
+      float rr = 1.f;
+      epilogue_prefetch<EPI>(p, row0 + lane, row0 + lane < p.M, n_blk, x0, x1, rr);
       // Warp-uniform outcome: tcgen05.ld below needs all 32 lanes converged.
       const bool ok = mbar_wait(&tfull[acc], acc_phase, ctl, 2 + q, kWaitAccFull);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
       es.row0 = row0;
+      es.begin_tile();
       epilogue_tile<EPI>(p, tbase, row0 + lane, row0 + lane < p.M, row0 / 32, n_blk, lane, es, &tmO1, &tmO2, x0,
-                         x1);
+                         x1, rr);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {

@@ -119,7 +119,8 @@ coda_status coda_selftest_wait_timeout(void* ws, uint64_t limit_ns, void* stream
 #define CODA_EPI_XENT_BWD 6   /* softmax - one-hot, dlogits */
 #define CODA_EPI_ROPE 7       /* rotary embedding (the QKV GEMM) */
 #define CODA_KERNEL_FOLD_GAIN 16          /* W2g = W2 diag(g) */
-#define CODA_KERNEL_RMS_ROWREDUCE 17      /* r from the partial sums of squares */
+#define CODA_KERNEL_RMS_ROWREDUCE 17      /* reserved: r is now formed in the gate/up GEMM's epilogue,
+                                             so no launch carries this id */
 #define CODA_KERNEL_SWIGLU_BWD_ROWSTAT 18 /* dA' = r [da | db] and the row coefficient c */
 #define CODA_KERNEL_COL_REDUCE 19         /* dg from its column partials */
 #define CODA_KERNEL_ROWCOEF_REDUCE 20     /* c from its row partials (MLP block backward) */
@@ -169,8 +170,9 @@ size_t coda_grg_fwd_workspace_bytes(int M, int K, int d, int N, int prefolded);
  * (toolin.ai §核心の洞察; kucoin (ru) §«В «Финале» спрятаны сокровища»):
  *   GEMM1 epilogue:  H = X W1^T + R (fp32 accumulate + fp32(R), stored bf16),
  *                    P[i, t] = sum_{j in tile t} bf16(H_ij)^2 (tiles of 256 columns)
- *   row reduce:      r_i = 1 / sqrt(sum_t P[i,t] / d + eps)            (fp32 [M])
- *   GEMM2 epilogue:  acc = H W2g^T with W2g = W2 diag(g);  a = r_i acc_gate,
+ *   GEMM2 epilogue:  r_i = 1 / sqrt(sum_t P[i,t] / d + eps) (the light row
+ *                    reduction, fp32 [M], stored once per row);
+ *                    acc = H W2g^T with W2g = W2 diag(g);  a = r_i acc_gate,
  *                    b = r_i acc_up;  Y = silu(a) * b  (bf16 [M, F]);
  *                    AB = [a | b] (bf16 [M, 2F]) saved for the backward.
  * Inputs:  X [M,K], W1 [d,K], R [M,d], g [d], W2 [N=2F, d] (all bf16).
@@ -410,7 +412,7 @@ coda_status coda_swiglu_bwd_unfused(const void* dOut, const void* X, const void*
  *
  * Computes exactly what coda_grg_fwd computes when given a pre-folded weight
  * (same kernels, same results): GEMM1 + residual + partial sums of squares,
- * the row reduce to r, GEMM2 + r + SwiGLU.  The caller passes every input and
+ * then GEMM2 forming r from them + SwiGLU.  The caller passes every input and
  * output (X [M,K], W1 [d,K], R [M,d], W2g = bf16(W2 diag(g)) [N,d] from
  * coda_fold_gain, H [M,d], r [M] fp32, Y [M,F], AB_or_null [M,N]); there is no
  * ws argument.  Its only scratch, the partial sums P[M, ceil(d/256)] and a

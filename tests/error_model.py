@@ -60,8 +60,10 @@ def _silu_derivs(a):
 
 
 def _mm_var(va, b2t):
-    """Variance of (A @ B) from the variance of A and the squares of B."""
-    return va @ b2t
+    """Variance of (A @ B) from the variance of A and the squares of B.  A
+    variance needs only a few significant digits, so the product runs in
+    float32 (twice as fast as float64 in BLAS)."""
+    return (np.asarray(va, dtype=np.float32) @ np.asarray(b2t, dtype=np.float32)).astype(np.float64)
 
 
 def _swiglu_fwd_var(a, b, va, vb):

@@ -34,4 +34,8 @@ def test_mlp_block_forward_backward(cuda_lib, M, K, d, F, eps):
     tag = f"block M={M} K={K} d={d} F={F}"
     ref = refs.mlp_block(t, eps)
     assert_tol(o["H"], ref["fs"]["H"], f"{tag} H")
-    refs.check_mlp_block(o, b, ref, tag)
+    si = refs.saved_inputs(ref)
+    bi = cuda_lib.mlp_block_bwd(td["dOut"], td["X"], td["W1"], si["H"], si["r"], si["AB"], si["Y"], td["g"],
+                                td["W2"], td["Wdown"])
+    torch.cuda.synchronize()
+    refs.check_mlp_block(o, b, bi, ref, tag)

@@ -79,14 +79,14 @@ def test_profile_hook_times_one_launch(cuda_lib):
 
 
 def test_profile_hook_times_every_kernel_of_a_step(cuda_lib):
-    """Pairs armed for all ten kernels of the block's forward and backward fire
+    """Pairs armed for all nine kernels of the block's forward and backward fire
     once each, in launch order (three for the plain-store GEMMs), and bracket
     non-overlapping stretches of the stream."""
     B = cuda_lib
     M, K, d, F = 1024, 1024, 1024, 2048
     t = synth.grg_inputs(M, K, d, F, seed=12)
     dv = {k: v.cuda() for k, v in t.items()}
-    ids = [B.KERNEL_FOLD_GAIN, B.EPI_RESID_RMS, B.KERNEL_RMS_ROWREDUCE, B.EPI_SWIGLU,
+    ids = [B.KERNEL_FOLD_GAIN, B.EPI_RESID_RMS, B.EPI_SWIGLU,
            B.KERNEL_SWIGLU_BWD_ROWSTAT, B.EPI_DN, B.KERNEL_COL_REDUCE, B.EPI_STORE, B.EPI_STORE, B.EPI_STORE]
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in ids]
     fo = B.grg_fwd(dv["X"], dv["W1"], dv["R"], dv["g"], dv["W2"], 1e-6)  # warm: allocations, tensor maps

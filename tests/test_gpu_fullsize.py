@@ -1,8 +1,10 @@
 """GPU parity at the full LLaMA-shaped workload sizes, in the launch configuration bench.py times.
 
 Every output element of every workload is compared with both oracles: the
-storage-precision fp64 oracle at the stated tolerance, and the pure fp64
-oracle at that tolerance widened by the deviation the method's bf16 storage
+storage-precision fp64 oracle at the stated tolerance (each entry point on
+the same inputs: a backward is also run on the saved tensors the oracle's
+forward produced), and the pure fp64 oracle, for the whole forward-backward
+chain, at that tolerance widened by the deviation the method's bf16 storage
 points produce in that element (tests/error_model.py).  No check allows
 outliers.  The host's BLAS runs each full oracle in tens of seconds.
 """
@@ -32,9 +34,20 @@ def _host(d):
 
 @pytest.mark.parametrize("name,M,K,d,F,eps,bwd", GRG_FULL, ids=[c[0] for c in GRG_FULL])
 def test_grg_full_size(cuda_lib, name, M, K, d, F, eps, bwd):
+    _grg_full(cuda_lib, name, M, K, d, F, eps, bwd, "weight")
+
+
+def test_grg_full_size_activation_gain(cuda_lib):
+    """The 7B block with the gain on the activation side: Hg = bf16(H*g) from
+    GEMM1's epilogue feeds GEMM2 (no fold), forward and backward."""
+    _grg_full(cuda_lib, "7B hg", 8192, 4096, 4096, 11008, 1e-6, True, "activation")
+
+
+def _grg_full(cuda_lib, name, M, K, d, F, eps, bwd, gain):
     t = synth.grg_inputs(M, K, d, F, seed=0)
     td = {k: v.cuda() for k, v in t.items()}
-    o = cuda_lib.grg_fwd(td["X"], td["W1"], td["R"], td["g"], td["W2"], eps)
+    fwd = cuda_lib.grg_fwd if gain == "weight" else cuda_lib.grg_fwd_hg
+    o = fwd(td["X"], td["W1"], td["R"], td["g"], td["W2"], eps)
     b = None
     if bwd:
         b = cuda_lib.grg_bwd(td["dY"], td["X"], td["W1"], o["H"], o["r"], o["AB"], td["g"], td["W2"])
@@ -43,30 +56,18 @@ def test_grg_full_size(cuda_lib, name, M, K, d, F, eps, bwd):
     assert st == 0, f"device status {st} detail {detail:#x}"
     go = _host(o)
     gb = _host(b) if b is not None else None
-    del o, b, td
+    del o, b
     torch.cuda.empty_cache()
-    ref = refs.grg(t, eps, bwd=bwd)
+    ref = refs.grg(t, eps, gain=gain, bwd=bwd)
     refs.check_grg_fwd(go, ref, name)
     if bwd:
-        refs.check_grg_bwd(gb, ref, name)
-    refs.release(ref)
-
-
-def test_grg_full_size_activation_gain(cuda_lib):
-    """The 7B block with the gain on the activation side: Hg = bf16(H*g) from
-    GEMM1's epilogue feeds GEMM2 (no fold), forward and backward."""
-    M, K, d, F, eps = 8192, 4096, 4096, 11008, 1e-6
-    t = synth.grg_inputs(M, K, d, F, seed=0)
-    td = {k: v.cuda() for k, v in t.items()}
-    o = cuda_lib.grg_fwd_hg(td["X"], td["W1"], td["R"], td["g"], td["W2"], eps)
-    b = cuda_lib.grg_bwd(td["dY"], td["X"], td["W1"], o["H"], o["r"], o["AB"], td["g"], td["W2"])
-    torch.cuda.synchronize()
-    go, gb = _host(o), _host(b)
-    del o, b, td
-    torch.cuda.empty_cache()
-    ref = refs.grg(t, eps, gain="activation")
-    refs.check_grg_fwd(go, ref, "7B hg")
-    refs.check_grg_bwd(gb, ref, "7B hg")
+        si = refs.saved_inputs(ref)
+        bi = cuda_lib.grg_bwd(td["dY"], td["X"], td["W1"], si["H"], si["r"], si["AB"], td["g"], td["W2"])
+        torch.cuda.synchronize()
+        gbi = _host(bi)
+        del bi, si
+        refs.check_grg_bwd(gb, gbi, ref, name)
+    del td
     refs.release(ref)
 
 
@@ -94,10 +95,15 @@ def test_swiglu_full_size(cuda_lib):
     b = cuda_lib.swiglu_bwd(td["dOut"], td["X"], td["Wgu"], td["Wdown"], o["Y"], o["AB"])
     torch.cuda.synchronize()
     go, gb = _host(o), _host(b)
-    del o, b, td
+    del o, b
     torch.cuda.empty_cache()
     ref = refs.swiglu(t)
-    refs.check_swiglu(go, gb, ref, "swiglu")
+    si = refs.saved_inputs(ref)
+    bi = cuda_lib.swiglu_bwd(td["dOut"], td["X"], td["Wgu"], td["Wdown"], si["Y"], si["AB"])
+    torch.cuda.synchronize()
+    gbi = _host(bi)
+    del bi, si, td
+    refs.check_swiglu(go, gb, gbi, ref, "swiglu")
     refs.release(ref)
 
 
@@ -111,8 +117,14 @@ def test_mlp_block_full_size(cuda_lib):
                                td["Wdown"])
     torch.cuda.synchronize()
     go, gb = _host(o), _host(b)
-    del o, b, td
+    del o, b
     torch.cuda.empty_cache()
     ref = refs.mlp_block(t, eps)
-    refs.check_mlp_block(go, gb, ref, "block 7B")
+    si = refs.saved_inputs(ref)
+    bi = cuda_lib.mlp_block_bwd(td["dOut"], td["X"], td["W1"], si["H"], si["r"], si["AB"], si["Y"], td["g"],
+                                td["W2"], td["Wdown"])
+    torch.cuda.synchronize()
+    gbi = _host(bi)
+    del bi, si, td
+    refs.check_mlp_block(go, gb, gbi, ref, "block 7B")
     refs.release(ref)

@@ -118,7 +118,11 @@ def test_grg_backward(cuda_lib, M, K, d, F, eps, with_dH_in):
                          dH_in=td.get("dH_in"))
     torch.cuda.synchronize()
     ref = refs.grg(t, eps, dH_in=with_dH_in)
-    refs.check_grg_bwd(b, ref, f"grg_bwd M={M} K={K} d={d} F={F} dH_in={with_dH_in}")
+    si = refs.saved_inputs(ref)
+    bi = cuda_lib.grg_bwd(td["dY"], td["X"], td["W1"], si["H"], si["r"], si["AB"], td["g"], td["W2"],
+                          dH_in=td.get("dH_in"))
+    torch.cuda.synchronize()
+    refs.check_grg_bwd(b, bi, ref, f"grg_bwd M={M} K={K} d={d} F={F} dH_in={with_dH_in}")
 
 
 def test_grg_structured_exact_indexing(cuda_lib):
@@ -174,7 +178,10 @@ def test_grg_zero_rows_forward_backward(cuda_lib):
     torch.cuda.synchronize()
     ref = refs.grg(t, eps)
     refs.check_grg_fwd(o, ref, "grg_fwd zero rows")
-    refs.check_grg_bwd(b, ref, "grg_bwd zero rows")
+    si = refs.saved_inputs(ref)
+    bi = cuda_lib.grg_bwd(td["dY"], td["X"], td["W1"], si["H"], si["r"], si["AB"], td["g"], td["W2"])
+    torch.cuda.synchronize()
+    refs.check_grg_bwd(b, bi, ref, "grg_bwd zero rows")
     r = o["r"].cpu().numpy()
     np.testing.assert_allclose(r[zero], 1.0 / np.sqrt(eps), rtol=1e-6)
     for name, v in (("H", o["H"]), ("Y", o["Y"]), ("AB", o["AB"]), ("dX", b["dX"]), ("dR", b["dR"])):
@@ -197,7 +204,11 @@ def test_swiglu_forward_backward(cuda_lib, M, d, F):
     o = cuda_lib.swiglu_fwd(td["X"], td["Wgu"], td["Wdown"])
     b = cuda_lib.swiglu_bwd(td["dOut"], td["X"], td["Wgu"], td["Wdown"], o["Y"], o["AB"])
     torch.cuda.synchronize()
-    refs.check_swiglu(o, b, refs.swiglu(t), f"swiglu M={M} d={d} F={F}")
+    ref = refs.swiglu(t)
+    si = refs.saved_inputs(ref)
+    bi = cuda_lib.swiglu_bwd(td["dOut"], td["X"], td["Wgu"], td["Wdown"], si["Y"], si["AB"])
+    torch.cuda.synchronize()
+    refs.check_swiglu(o, b, bi, ref, f"swiglu M={M} d={d} F={F}")
 
 
 def test_status_word_stays_clear(cuda_lib):
@@ -223,7 +234,10 @@ def test_grg_forward_activation_gain(cuda_lib, M, K, d, F, eps):
     ref = refs.grg(t, eps, gain="activation")
     refs.check_grg_fwd(o, ref, tag)
     np.testing.assert_array_equal(f64(o["Hg"]), O.round_bf16(f64(o["H"]) * f64(t["g"])[None, :]))
-    refs.check_grg_bwd(b, ref, f"{tag} bwd")
+    si = refs.saved_inputs(ref)
+    bi = cuda_lib.grg_bwd(td["dY"], td["X"], td["W1"], si["H"], si["r"], si["AB"], td["g"], td["W2"])
+    torch.cuda.synchronize()
+    refs.check_grg_bwd(b, bi, ref, f"{tag} bwd")
 
 
 def test_run_to_run_bit_reproducible(cuda_lib):
