@@ -211,17 +211,6 @@ int raster_budget_mb() {
   }();
   return v;
 }
-// Distance, in k-blocks, at which the TMA producer prefetches operand boxes
-// into L2 ahead of its loads (CODA_L2_PREFETCH; 0 turns prefetching off).
-int l2_prefetch_stages() {
-  static const int v = [] {
-    const char* e = std::getenv("CODA_L2_PREFETCH");
-    const int x = e ? std::atoi(e) : 0;
-    return x > 0 ? std::min(x, 64) : 0;
-  }();
-  return v;
-}
-
 int pick_group(long long a_rows, long long b_rows, long long K, int num_m, int num_n, bool pair, int num_sms) {
   const int units = pair ? num_sms / 2 : num_sms;
   int side = 1;
@@ -283,7 +272,6 @@ coda_status launch_gemm_mode(const CUtensorMap& ta, const CUtensorMap& tb, GemmP
     return CODA_ERR_CUDA;
   p.kernel_id = (uint32_t)(slot + 1);
   p.wait_limit_ns = g_wait_limit_ns.load();
-  p.prefetch_stages = l2_prefetch_stages();
   if (p.group_m == 0) p.group_m = 1;
   const int tiles = p.num_m_tiles * p.num_n_tiles;
   const int units = std::min(tiles, di.max_clusters[slot]);  // persistent: one tile stream per CTA (pair)

@@ -79,7 +79,6 @@ struct GemmParams {
   int rot_cols;                 // ROPE: columns [0, rot_cols) are rotated (q and k heads)
   int seq_len;                  // ROPE: position = row % seq_len
   float rope_k;                 // ROPE: -2 log2(base) / head_dim, so inv_freq_j = 2^(j * rope_k)
-  int prefetch_stages;          // L2 prefetch distance of the producer in stages (0: none)
   float inv_d;                  // SWIGLU with part: 1 / d of the RMSNorm mean
   float eps;                    // SWIGLU with part: the RMSNorm eps
   uint32_t* status;
@@ -527,40 +526,6 @@ struct TileCfg {
   static constexpr int CTAS = PAIR ? 2 : 1;
 };
 
-// L2 prefetch of the operand boxes this CTA loads for k-block kb of `tile`:
-// the same boxes as the producer's loads, issued prefetch_stages stages ahead
-// so that a miss in L2 is served from DRAM while the ring still holds earlier
-// stages.
-template <int EPI, bool A_MN, bool B_MN, bool PAIR>
-__device__ __forceinline__ void prefetch_stage(const CUtensorMap* tmA, const CUtensorMap* tmB, const GemmParams& p,
-                                               int tile, int kb, uint32_t rank) {
-  using C = TileCfg<PAIR>;
-  int m_blk, n_blk;
-  tile_coords(tile, p.num_m_tiles, p.num_n_tiles, p.group_m, m_blk, n_blk);
-  const int a_row = m_blk * C::TILE_M + (int)rank * 128;
-  const int k0 = kb * BK;
-  if constexpr (!A_MN) {
-    tma_prefetch_2d(tmA, k0, a_row);
-  } else {
-#pragma unroll
-    for (int c = 0; c < 2; ++c) tma_prefetch_2d(tmA, a_row + c * 64, k0);
-  }
-  if constexpr (EPI == EPI_SWIGLU) {
-    if constexpr (PAIR) {
-      tma_prefetch_2d(tmB, k0, (rank ? p.split : 0) + n_blk * (BN / 2));
-    } else {
-      tma_prefetch_2d(tmB, k0, n_blk * (BN / 2));
-      tma_prefetch_2d(tmB, k0, p.split + n_blk * (BN / 2));
-    }
-  } else if constexpr (!B_MN) {
-    tma_prefetch_2d(tmB, k0, n_blk * BN + (PAIR ? (int)rank * 128 : 0));
-  } else {
-    constexpr int chunks = PAIR ? 2 : BN / 64;
-#pragma unroll
-    for (int c = 0; c < chunks; ++c) tma_prefetch_2d(tmB, n_blk * BN + (PAIR ? (int)rank * 128 : 0) + c * 64, k0);
-  }
-}
-
 template <int EPI, bool A_MN, bool B_MN, bool PAIR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -636,24 +601,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      // L2 prefetch cursor, prefetch_stages k-blocks ahead of the loads.
-      int pf_tile = first_tile, pf_kb = p.prefetch_stages;
-      while (pf_kb >= p.k_blocks && p.prefetch_stages > 0) {
-        pf_kb -= p.k_blocks;
-        pf_tile += tile_step;
-      }
       for (int tile = first_tile; tile < num_tiles && ok; tile += tile_step) {
         int m_blk, n_blk;
         tile_coords(tile, p.num_m_tiles, p.num_n_tiles, p.group_m, m_blk, n_blk);
         const int a_row = m_blk * C::TILE_M + (int)rank * 128;
         for (int kb = 0; kb < p.k_blocks; ++kb) {
-          if (p.prefetch_stages > 0 && pf_tile < num_tiles) {
-            prefetch_stage<EPI, A_MN, B_MN, PAIR>(&tmA, &tmB, p, pf_tile, pf_kb, rank);
-            if (++pf_kb == p.k_blocks) {
-              pf_kb = 0;
-              pf_tile += tile_step;
-            }
-          }
           if (!mbar_wait(&empty[stage], phase ^ 1u, ctl, 0, kWaitEmpty)) {
             ok = false;
             break;
