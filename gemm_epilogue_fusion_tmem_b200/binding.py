@@ -91,6 +91,8 @@ def library() -> ctypes.CDLL:
             "coda_grg_fwd_unfused": (I, [P] * 10 + [I, I, I, I, F, P, S, P]),
             "coda_grg_bwd_unfused_workspace_bytes": (S, [I, I, I, I]),
             "coda_grg_bwd_unfused": (I, [P] * 15 + [I, I, I, I, P, S, P]),
+            "coda_grg_fwd_prefolded_static": (I, [P] * 8 + [I, I, I, I, F, P]),
+            "coda_static_status_query": (I, [P, ctypes.POINTER(ctypes.c_uint32)]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)
@@ -104,7 +106,7 @@ def library() -> ctypes.CDLL:
 
 # Host-side entry points that enqueue no GPU work get no NVTX range.
 _UNRANGED = {"coda_status_string", "coda_version", "coda_set_wait_limit_ns", "coda_profile_arm",
-             "coda_status_query"}
+             "coda_status_query", "coda_static_status_query"}
 
 
 class _Ranged:
@@ -126,6 +128,13 @@ class _Ranged:
 
     def __getattr__(self, key):
         return getattr(self._fn, key)
+
+    def __setattr__(self, key, value):
+        # restype / argtypes set by a caller go to the ctypes function itself
+        if key in self.__slots__:
+            object.__setattr__(self, key, value)
+        else:
+            setattr(self._fn, key, value)
 
 
 def _status_string(status: int) -> str:
@@ -309,6 +318,44 @@ def grg_fwd(X, W1, R, g, W2, eps: float, W2g=None, save_ab: bool = True, out: di
                             _ptr(o["r"]), _ptr(o["Y"]), _ptr(AB), M, K, d, N, float(eps),
                             ws.ptr(), ws.nbytes, _stream()), "coda_grg_fwd")
     return o
+
+
+def grg_fwd_prefolded_static(X, W1, R, W2g, eps: float, save_ab: bool = True, out: dict | None = None) -> dict:
+    """The forward for callers that cannot allocate device memory: the same
+    kernels as grg_fwd given a pre-folded W2g, with the scratch in the
+    library's static device array (no workspace).  Outputs are allocated here
+    unless passed in `out`; a caller that must not allocate passes them all.
+    Calls that overlap on the GPU share the static array and must be
+    serialised.  Returns H, r, Y, AB."""
+    lib = library()
+    M, K = X.shape
+    d = W1.shape[0]
+    N = W2g.shape[0]
+    F = N // 2
+    _req(X, "X"), _req(W1, "W1", shape=(d, K)), _req(R, "R", shape=(M, d)), _req(W2g, "W2g", shape=(N, d))
+    o = dict(out or {})
+    dev = X.device
+    for k, shape, dt in (("H", (M, d), torch.bfloat16), ("r", (M,), torch.float32), ("Y", (M, F), torch.bfloat16)):
+        if k not in o:
+            o[k] = torch.empty(*shape, dtype=dt, device=dev)
+        _req(o[k], k, dt, shape)
+    if save_ab and "AB" not in o:
+        o["AB"] = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    AB = o.get("AB") if save_ab else None
+    if AB is not None:
+        _req(AB, "AB", shape=(M, N))
+    _check(lib.coda_grg_fwd_prefolded_static(_ptr(X), _ptr(W1), _ptr(R), _ptr(W2g), _ptr(o["H"]), _ptr(o["r"]),
+                                             _ptr(o["Y"]), _ptr(AB), M, K, d, N, float(eps), _stream()),
+           "coda_grg_fwd_prefolded_static")
+    return o
+
+
+def static_status() -> tuple[int, int]:
+    """Synchronise the current stream and return (status, detail) of the last
+    grg_fwd_prefolded_static call on the current device."""
+    detail = ctypes.c_uint32(0)
+    st = library().coda_static_status_query(_stream(), ctypes.byref(detail))
+    return int(st), int(detail.value)
 
 
 def grg_fwd_hg(X, W1, R, g, W2, eps: float, save_ab: bool = True, keep_hg: bool = False, out: dict | None = None,

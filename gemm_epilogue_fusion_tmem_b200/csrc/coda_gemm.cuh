@@ -694,8 +694,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           // Free the stage (in both CTAs of a pair) once these MMAs have read it.
           if constexpr (PAIR) {
-            umma_commit_pair(mapa_shared(smem_u32(&empty[stage]), 0));
-            umma_commit_pair(mapa_shared(smem_u32(&empty[stage]), 1));
+            umma_commit_pair_both(&empty[stage]);
           } else {
             umma_commit(&empty[stage]);
           }
@@ -707,8 +706,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!ok) break;
         // Accumulator ready for the epilogue warps (of both CTAs of a pair).
         if constexpr (PAIR) {
-          umma_commit_pair(mapa_shared(smem_u32(&tfull[acc]), 0));
-          umma_commit_pair(mapa_shared(smem_u32(&tfull[acc]), 1));
+          umma_commit_pair_both(&tfull[acc]);
         } else {
           umma_commit(&tfull[acc]);
         }

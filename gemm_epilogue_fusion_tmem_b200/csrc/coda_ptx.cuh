@@ -333,6 +333,18 @@ __device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t a_desc,
       : "memory");
 }
 
+// Arrive once on the mbarrier at shared offset `bar` in both CTAs of the pair
+// (CTA mask 0b11) when all prior pair MMAs of this thread complete.  One
+// multicast commit instead of one commit per CTA: in a same-box A/B the
+// per-CTA pair of commits cost the tensor pipe 4-12 % (the commits are
+// ordered with the MMAs they track).
+__device__ __forceinline__ void umma_commit_pair_both(const uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+                   smem_u32(bar)),
+               "h"((uint16_t)3)
+               : "memory");
+}
+
 // Arrive once on the mbarrier at `bar_cluster_addr` when all prior pair MMAs of this thread complete.
 __device__ __forceinline__ void umma_commit_pair(uint32_t bar_cluster_addr) {
   asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
