@@ -33,6 +33,8 @@ sys.path.insert(0, ROOT)
 METRIC = "fused GEMM-RMSNorm-GEMM fwd+bwd TFLOP/s and % of B200 bf16 tensor peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 DENSE_BF16_FLOP_PER_SM_CLK = 8192  # tcgen05 dense bf16: 4096 multiply-adds per SM per clock
+INTERLEAVED = ("10 rounds of alternating bursts of at least 5 steps each, the order swapped every round, "
+               "median ms per step of each")
 
 WORKLOADS = {
     "tiny": ("grg", dict(M=256, K=512, d=512, F=1024, eps=1e-6), True),
@@ -484,19 +486,21 @@ def _time_loop(fn, steps, warmup, device, world, barrier):
     return max_over_ranks(e0.elapsed_time(e1), device, world)
 
 
-def _time_interleaved(fa, fb, steps, warmup, device, world, barrier, rounds=6):
-    """Median ms per call of fa and of fb, timed in alternating bursts (fa, fb,
-    fa, fb, ...) so that both see the same thermal and power-cap drift; each
-    burst is max over ranks."""
+def _time_interleaved(fa, fb, steps, warmup, device, world, barrier, rounds=10):
+    """Median ms per call of fa and of fb, timed in alternating bursts of at
+    least 5 calls, the order swapped every round (fa fb, fb fa, ...), so that
+    both see the same thermal and power-cap drift and neither always runs
+    first; each burst is max over ranks."""
     import statistics
-    per = max(1, steps // rounds)
+    per = max(5, steps // 4)
     for _ in range(max(warmup, 3)):
         fa()
         fb()
     ta, tb = [], []
-    for _ in range(rounds):
-        ta.append(_time_loop(fa, per, None, device, world, barrier) / per)
-        tb.append(_time_loop(fb, per, None, device, world, barrier) / per)
+    for i in range(rounds):
+        order = ((fa, ta), (fb, tb)) if i % 2 == 0 else ((fb, tb), (fa, ta))
+        for fn, acc in order:
+            acc.append(_time_loop(fn, per, None, device, world, barrier) / per)
     return statistics.median(ta), statistics.median(tb)
 
 
@@ -561,7 +565,7 @@ def grg_extra(name, a, device, world, barrier):
         raise SystemExit(f"bench.py: device status {status} detail {detail:#x} in the {name} extra")
     rate = lambda ms: round(replica_throughput(flops, 1, world, ms), 2)  # noqa: E731
     out = {"config": _describe(name, kind, s, bwd), "flops_per_step": flops,
-           "timing": "alternating bursts (fused, unfused, fused, ...), median ms per step of each",
+           "timing": INTERLEAVED,
            "fused_folded_gain": {"ms_per_step": round(f_ms, 4), "value": rate(f_ms),
                                  "frac_of_burst": round(rate(f_ms) / world / burst, 4),
                                  "unfused_ms_per_step": round(u_ms, 4), "speedup_vs_unfused": round(u_ms / f_ms, 4),
@@ -907,7 +911,7 @@ def run_coda(a):
         variants["activation_gain"] = {"ms_per_step": round(h_ms, 4),
                                        "value": round(replica_throughput(flops, 1, world, h_ms), 2),
                                        "fused_ms_per_step": round(f_ms, 4),
-                                       "timing": "alternating bursts with the folded-gain step, medians",
+                                       "timing": INTERLEAVED + " (against the folded-gain step)",
                                        "what": "coda_grg_fwd_hg: GEMM1 stores H*g, GEMM2 reads W2 unfolded"}
         del hws
 
@@ -925,7 +929,7 @@ def run_coda(a):
         variants["cuda_graph"] = {"ms_per_step": round(g_ms, 4),
                                   "value": round(replica_throughput(flops, 1, world, g_ms), 2),
                                   "eager_ms_per_step": round(e_ms, 4),
-                                  "timing": "alternating bursts with the eager step, medians",
+                                  "timing": INTERLEAVED + " (against the eager step)",
                                   "what": "the same step captured once with torch.cuda.graph and replayed"}
         del graph
     except RuntimeError as err:  # capture not possible: report it instead of a number
@@ -943,8 +947,7 @@ def run_coda(a):
         unfused = {"ms_per_step": round(u_ms, 4),
                    "value": round(replica_throughput(flops, 1, world, u_ms), 2), "unit": "TFLOP/s",
                    "fused_ms_per_step": round(f_ms, 4), "fused_speedup": round(u_ms / f_ms, 4),
-                   "gpu_launches_per_step": ulaunch, "timing": "alternating bursts of fused and unfused steps, "
-                                                               "median ms per step of each",
+                   "gpu_launches_per_step": ulaunch, "timing": INTERLEAVED,
                    "what": "same GEMM kernels with plain stores; residual add, RMSNorm, SwiGLU and their backward "
                            "as separate HBM-round-trip kernels"}
         for dname in ("fwd", "bwd"):

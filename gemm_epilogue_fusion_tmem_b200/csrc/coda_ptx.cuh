@@ -362,12 +362,16 @@ namespace coda {
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
-// 2-D tiled bulk tensor store from this CTA's shared memory; rows/columns
-// outside the tensor are not written.  x is the innermost coordinate.
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, const void* smem_src, int x, int y) {
-  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+// 2-D tiled bulk tensor store from this CTA's shared memory with an L2 cache
+// policy (evict-first for the epilogue's outputs, which the kernel never reads
+// back: they leave L2 before the operand panels that the concurrent tiles are
+// still reading); rows/columns outside the tensor are not written.  x is the
+// innermost coordinate.
+__device__ __forceinline__ void tma_store_2d_hint(const CUtensorMap* m, const void* smem_src, int x, int y,
+                                                  uint64_t policy) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%2, %3}], [%1], %4;" ::"l"(
                    reinterpret_cast<uint64_t>(m)),
-               "r"(smem_u32(smem_src)), "r"(x), "r"(y)
+               "r"(smem_u32(smem_src)), "r"(x), "r"(y), "l"(policy)
                : "memory");
 }
 __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
