@@ -67,6 +67,19 @@ def test_static_scratch_forward_matches_workspace_forward(cuda_lib):
                                f"static fwd seed {seed}")
 
 
+def test_static_scratch_forward_through_the_binding(cuda_lib):
+    """The Python binding's wrapper calls the same entry point: bit-identical to
+    coda_grg_fwd with the same pre-folded weight, and the status word reads 0."""
+    M, K, d, F, eps = 256, 512, 512, 1024, 1e-6
+    t = {k: v.cuda() for k, v in synth.grg_inputs(M, K, d, F, seed=13).items()}
+    W2g = cuda_lib.fold_gain(t["W2"], t["g"])
+    ref = cuda_lib.grg_fwd(t["X"], t["W1"], t["R"], t["g"], t["W2"], eps, W2g=W2g)
+    got = cuda_lib.grg_fwd_prefolded_static(t["X"], t["W1"], t["R"], W2g, eps)
+    assert cuda_lib.static_status() == (0, 0)
+    for name in ("H", "r", "Y", "AB"):
+        assert torch.equal(got[name], ref[name]), name
+
+
 def test_static_scratch_forward_rejects_oversized_shapes(cuda_lib):
     lib = cuda_lib.library()
     fn = lib.coda_grg_fwd_prefolded_static
