@@ -25,13 +25,16 @@ __global__ void fold_gain_kernel(const __nv_bfloat16* __restrict__ W2, const __n
   long long v = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   int jv = (int)(v % dv);  // column vector of v; advanced by S mod dv per step
   for (; v < n_vec8; v += FOLD_UNROLL * S) {
-    uint4 w[FOLD_UNROLL];
-    int jj[FOLD_UNROLL];
+    // The step's loads of W2 and of g are independent of its stores, so all
+    // are issued first.  g (d values, reused by every row) goes through L1.
+    uint4 w[FOLD_UNROLL], gq[FOLD_UNROLL];
 #pragma unroll
     for (int u = 0; u < FOLD_UNROLL; ++u) {
       const long long vu = v + u * S;
-      jj[u] = jv;
-      if (vu < n_vec8) w[u] = ldg_nc_v4(W2 + vu * 8);
+      if (vu < n_vec8) {
+        w[u] = ldg_nc_v4(W2 + vu * 8);
+        gq[u] = ldg_nc_v4_l1(g + jv * 8);
+      }
       jv += s_mod;
       if (jv >= dv) jv -= dv;
     }
@@ -41,7 +44,7 @@ __global__ void fold_gain_kernel(const __nv_bfloat16* __restrict__ W2, const __n
       if (vu >= n_vec8) break;
       float f[8], gg[8];
       unpack8(w[u], f);
-      unpack8(ldg_nc_v4(g + jj[u] * 8), gg);
+      unpack8(gq[u], gg);
 #pragma unroll
       for (int i = 0; i < 8; ++i) f[i] *= gg[i];
       stg_v4(W2g + vu * 8, pack8(f));
