@@ -101,8 +101,43 @@ EncodeTiledFn encode_fn() {
 // Row-major bf16 matrix [rows][cols] (cols contiguous), swizzled boxes of
 // box_cols x box_rows (128-byte swizzle unless given); out-of-range elements
 // load as zero and are not written by stores.
+// Encoded tensor maps, cached per host thread.  A map is a pure function of
+// the arguments below, so a hit returns exactly what encoding would; it saves
+// the driver call on repeated launches over the same tensors, which is most
+// of the host time of a launch-bound step.
+struct TmapKey {
+  const void* base;
+  long long rows, cols;
+  int box_cols, box_rows, swizzle;
+  bool operator==(const TmapKey& o) const {
+    return base == o.base && rows == o.rows && cols == o.cols && box_cols == o.box_cols &&
+           box_rows == o.box_rows && swizzle == o.swizzle;
+  }
+};
+struct TmapSlot {
+  TmapKey key;
+  CUtensorMap map;
+  bool valid;
+};
+constexpr int kTmapCacheSlots = 64;
+thread_local TmapSlot t_tmap_cache[kTmapCacheSlots];
+
+int tmap_slot(const TmapKey& k) {
+  uint64_t h = reinterpret_cast<uintptr_t>(k.base) >> 4;
+  for (uint64_t v : {(uint64_t)k.rows, (uint64_t)k.cols, (uint64_t)k.box_cols, (uint64_t)k.box_rows,
+                     (uint64_t)k.swizzle})
+    h = (h ^ v) * 0x9E3779B97F4A7C15ull;
+  return (int)((h >> 32) % kTmapCacheSlots);
+}
+
 bool make_tmap(CUtensorMap* m, const void* base, long long rows, long long cols, int box_cols, int box_rows,
                CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
+  const TmapKey key{base, rows, cols, box_cols, box_rows, (int)swizzle};
+  TmapSlot& slot = t_tmap_cache[tmap_slot(key)];
+  if (slot.valid && slot.key == key) {
+    *m = slot.map;
+    return true;
+  }
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return false;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
@@ -112,7 +147,11 @@ bool make_tmap(CUtensorMap* m, const void* base, long long rows, long long cols,
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  if (r != CUDA_SUCCESS) return false;
+  slot.key = key;
+  slot.map = *m;
+  slot.valid = true;
+  return true;
 }
 
 // Operand with logical shape [mn, k].  K-major storage is [mn][k]; MN-major
