@@ -153,50 +153,80 @@ __global__ void __launch_bounds__(COLRED_THREADS)
   }
 }
 
-// Cross-entropy row reduce, one warp per row: merge the tiles' (max, sum exp)
-// partials, lse = max + log(sum), loss = lse - target logit (the target logit
-// is NaN when the target was out of range, so the loss is too).
 // Inverse RoPE of the q/k gradient (rotation by -pos * base^(-2j/hd)) and a
-// copy of the v gradient, 8 pairs (or 8 v columns) per thread:
-// dpre = R(pos)^T dQKV, the A operand of the backward GEMMs.
+// copy of the v gradient: dpre = R(pos)^T dQKV, the A operand of the backward
+// GEMMs.  A rotation item is one row, one slice of 8 pairs (j0 .. j0 + 7) and
+// up to ROPE_HEADS rotated heads; the heads share the slice's angles, so its
+// 8 sines and cosines are computed once for all of them, and the heads' loads
+// are issued in groups of 4 before any store.  A copy item is 8 v columns.
+constexpr int ROPE_HEADS = 8;
 __global__ void rope_unrotate_kernel(const __nv_bfloat16* __restrict__ dq, __nv_bfloat16* __restrict__ dpre,
                                      int M, int ncols, int head_dim, int rot_cols, int seq_len, float rope_k) {
   griddep_wait();
   const int half = head_dim / 2;
-  const int rot_items = (rot_cols / head_dim) * (half / 8);
-  const int per_row = rot_items + (ncols - rot_cols) / 8;
-  const long long total = (long long)M * per_row;
+  const int slices = half / 8;
+  const int rot_heads = rot_cols / head_dim;
+  const int groups = (rot_heads + ROPE_HEADS - 1) / ROPE_HEADS;
+  const long long rot_total = (long long)M * slices * groups;
+  const int copy_per_row = (ncols - rot_cols) / 8;
+  const long long total = rot_total + (long long)M * copy_per_row;
   const long long stride = (long long)gridDim.x * blockDim.x;
   for (long long it = (long long)blockIdx.x * blockDim.x + threadIdx.x; it < total; it += stride) {
-    const int row = (int)(it / per_row);
-    const int k = (int)(it - (long long)row * per_row);
-    const size_t base = (size_t)row * ncols;
-    if (k >= rot_items) {
-      const int c = rot_cols + (k - rot_items) * 8;
-      stg_v4(dpre + base + c, ldg_nc_v4(dq + base + c));
+    if (it >= rot_total) {
+      const long long ci = it - rot_total;
+      const int row = (int)(ci / copy_per_row);
+      const size_t off = (size_t)row * ncols + rot_cols + (size_t)(ci - (long long)row * copy_per_row) * 8;
+      stg_v4(dpre + off, ldg_nc_v4(dq + off));
       continue;
     }
-    const int h = k / (half / 8);
-    const int j0 = (k - h * (half / 8)) * 8;
-    const int c1 = h * head_dim + j0;
-    float x1[8], x2[8];
-    unpack8(ldg_nc_v4(dq + base + c1), x1);
-    unpack8(ldg_nc_v4(dq + base + c1 + half), x2);
+    // it = (row * groups + group) * slices + slice: neighbouring threads take
+    // neighbouring slices of one head group, so their 16-byte accesses abut.
+    const int sl = (int)(it % slices);
+    const long long rg = it / slices;
+    const int grp = (int)(rg % groups);
+    const int row = (int)(rg / groups);
+    const int j0 = sl * 8;
     const float pos = (float)(row % seq_len);
+    float sn[8], cs[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      float sn, cs;
-      sincosf(pos * exp2f((float)(j0 + i) * rope_k), &sn, &cs);
-      const float y1 = x1[i] * cs + x2[i] * sn;
-      const float y2 = x2[i] * cs - x1[i] * sn;
-      x1[i] = y1;
-      x2[i] = y2;
+    for (int i = 0; i < 8; ++i) sincosf(pos * exp2f((float)(j0 + i) * rope_k), &sn[i], &cs[i]);
+    const size_t base = (size_t)row * ncols + j0;
+    const int h_end = min(rot_heads, (grp + 1) * ROPE_HEADS);
+#pragma unroll 1
+    for (int h0 = grp * ROPE_HEADS; h0 < h_end; h0 += 4) {
+      uint4 q1[4], q2[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        if (h0 + k < h_end) {
+          const size_t c1 = base + (size_t)(h0 + k) * head_dim;
+          q1[k] = ldg_nc_v4(dq + c1);
+          q2[k] = ldg_nc_v4(dq + c1 + half);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        if (h0 + k >= h_end) break;
+        float x1[8], x2[8];
+        unpack8(q1[k], x1);
+        unpack8(q2[k], x2);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float y1 = x1[i] * cs[i] + x2[i] * sn[i];
+          const float y2 = x2[i] * cs[i] - x1[i] * sn[i];
+          x1[i] = y1;
+          x2[i] = y2;
+        }
+        const size_t c1 = base + (size_t)(h0 + k) * head_dim;
+        stg_v4(dpre + c1, pack8(x1));
+        stg_v4(dpre + c1 + half, pack8(x2));
+      }
     }
-    stg_v4(dpre + base + c1, pack8(x1));
-    stg_v4(dpre + base + c1 + half, pack8(x2));
   }
 }
 
+// Cross-entropy row reduce, one warp per row: merge the tiles' (max, sum exp)
+// partials, lse = max + log(sum), loss = lse - target logit (the target logit
+// is NaN when the target was out of range, so the loss is too).
 __device__ __forceinline__ void lse_merge(float& m, float& s, float om, float os) {
   if (om == -INFINITY) return;
   if (m == -INFINITY) {

@@ -444,26 +444,33 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tbas
       es.flush();
     }
   } else if constexpr (EPI == EPI_ROPE) {
+    // Every head of the tile turns its (j, j + hd/2) pairs by the same angles
+    // pos * inv_freq_j, so the sines and cosines of each 32-frequency slice
+    // are computed once per row and applied to all the tile's rotated heads
+    // (heads run q, k, v, so if the tile's first head is not rotated, none is).
     const int n0 = n_blk * BN;
     const float pos = (float)(row % p.seq_len);
     const int half = p.head_dim / 2;
+    const bool any_rot = n0 < p.rot_cols;
 #pragma unroll 1
-    for (int h0 = 0; h0 < BN; h0 += p.head_dim) {
-      const int col0 = n0 + h0;
-      if (col0 >= p.N) break;
-      const bool rot = col0 < p.rot_cols;
+    for (int c = 0; c < half; c += 32) {
+      float sn[32], cs[32];
+      if (any_rot) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) sincosf(pos * exp2f((float)(c + i) * p.rope_k), &sn[i], &cs[i]);
+      }
 #pragma unroll 1
-      for (int c = 0; c < half; c += 32) {
+      for (int h0 = 0; h0 < BN; h0 += p.head_dim) {
+        const int col0 = n0 + h0;
+        if (col0 >= p.N) break;
         float x1[32], x2[32];
         tmem_ld32(tbase + h0 + c, x1);
         tmem_ld32(tbase + h0 + half + c, x2);
-        if (rot) {
-#pragma unroll 4
+        if (col0 < p.rot_cols) {
+#pragma unroll
           for (int i = 0; i < 32; ++i) {
-            float sn, cs;
-            sincosf(pos * exp2f((float)(c + i) * p.rope_k), &sn, &cs);
-            const float y1 = x1[i] * cs - x2[i] * sn;
-            const float y2 = x2[i] * cs + x1[i] * sn;
+            const float y1 = x1[i] * cs[i] - x2[i] * sn[i];
+            const float y2 = x2[i] * cs[i] + x1[i] * sn[i];
             x1[i] = y1;
             x2[i] = y2;
           }
