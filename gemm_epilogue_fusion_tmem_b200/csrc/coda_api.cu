@@ -1120,7 +1120,7 @@ coda_status coda_qkv_rope_bwd(const void* dQKV, const void* X, const void* Wqkv,
   __nv_bfloat16* dpre = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(ws) + kStatusBytes);
   const int rot_cols = (n_q + n_kv) * head_dim;
   const long long rot_groups = cdiv(rot_cols / head_dim, ROPE_HEADS);
-  const long long items = (long long)M * (rot_groups * (head_dim / 16) + (ncols - rot_cols) / 8);
+  const long long items = (long long)M * (rot_groups * (head_dim / 16) + (ncols - rot_cols) / ROPE_COPY_COLS);
   CODA_TRY(launch_status(launch_ex(rope_unrotate_kernel, dim3(ew_grid(items)), dim3(256), 0, s, 1, cbf(dQKV),
                                    dpre, M, ncols, head_dim, rot_cols, seq_len, rope_k(head_dim, base))));
   CODA_TRY(gemm_store(dpre, Wqkv, dX, M, d, ncols, false, true, nullptr, ws, s));

@@ -158,8 +158,10 @@ __global__ void __launch_bounds__(COLRED_THREADS)
 // GEMMs.  A rotation item is one row, one slice of 8 pairs (j0 .. j0 + 7) and
 // up to ROPE_HEADS rotated heads; the heads share the slice's angles, so its
 // 8 sines and cosines are computed once for all of them, and the heads' loads
-// are issued in groups of 4 before any store.  A copy item is 8 v columns.
+// are issued in groups of 4 before any store.  A copy item is 32 v columns,
+// four 16-byte loads issued before their stores.
 constexpr int ROPE_HEADS = 8;
+constexpr int ROPE_COPY_COLS = 32;
 __global__ void rope_unrotate_kernel(const __nv_bfloat16* __restrict__ dq, __nv_bfloat16* __restrict__ dpre,
                                      int M, int ncols, int head_dim, int rot_cols, int seq_len, float rope_k) {
   griddep_wait();
@@ -168,15 +170,20 @@ __global__ void rope_unrotate_kernel(const __nv_bfloat16* __restrict__ dq, __nv_
   const int rot_heads = rot_cols / head_dim;
   const int groups = (rot_heads + ROPE_HEADS - 1) / ROPE_HEADS;
   const long long rot_total = (long long)M * slices * groups;
-  const int copy_per_row = (ncols - rot_cols) / 8;
+  const int copy_per_row = (ncols - rot_cols) / ROPE_COPY_COLS;  // v heads are multiples of 64 columns
   const long long total = rot_total + (long long)M * copy_per_row;
   const long long stride = (long long)gridDim.x * blockDim.x;
   for (long long it = (long long)blockIdx.x * blockDim.x + threadIdx.x; it < total; it += stride) {
     if (it >= rot_total) {
       const long long ci = it - rot_total;
       const int row = (int)(ci / copy_per_row);
-      const size_t off = (size_t)row * ncols + rot_cols + (size_t)(ci - (long long)row * copy_per_row) * 8;
-      stg_v4(dpre + off, ldg_nc_v4(dq + off));
+      const size_t off =
+          (size_t)row * ncols + rot_cols + (size_t)(ci - (long long)row * copy_per_row) * ROPE_COPY_COLS;
+      uint4 v[ROPE_COPY_COLS / 8];
+#pragma unroll
+      for (int k = 0; k < ROPE_COPY_COLS / 8; ++k) v[k] = ldg_nc_v4(dq + off + 8 * k);
+#pragma unroll
+      for (int k = 0; k < ROPE_COPY_COLS / 8; ++k) stg_v4(dpre + off + 8 * k, v[k]);
       continue;
     }
     // it = (row * groups + group) * slices + slice: neighbouring threads take
