@@ -25,6 +25,7 @@ import os
 import statistics
 import subprocess
 import sys
+import threading
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -197,11 +198,61 @@ CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.a
 
 
 class ClockSampler:
-    def __init__(self, device_index: int):
+    """Samples this process's GPU while the `with` block runs: SM clock, its
+    maximum, power and the active clock-event reasons.  Every 10 ms through
+    NVML on a thread (the device found by its UUID), so that even a region of
+    a few tens of milliseconds gets several samples; every 50 ms through
+    nvidia-smi when NVML cannot read the device.  Only reads counters."""
+
+    # NVML clock-event reason bits, named as nvidia-smi names them.
+    REASON_BITS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+                   ("sw_power_cap", 0x4))
+
+    def __init__(self, device_index: int, interval_s: float = 0.01):
         self.idx = device_index
+        self.interval = interval_s
         self.proc = None
+        self.thread = None
+        self.rows = []  # (sm MHz, max sm MHz, power W, reason bits) per NVML sample
+        self.out = ""
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            import torch
+            u = str(torch.cuda.get_device_properties(self.idx).uuid)
+            return pynvml.nvmlDeviceGetHandleByUUID(u if u.startswith("GPU-") else "GPU-" + u)
+        except Exception:
+            ids = [x.strip() for x in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if x.strip()]
+            phys = int(ids[self.idx]) if self.idx < len(ids) and ids[self.idx].isdigit() else self.idx
+            return pynvml.nvmlDeviceGetHandleByIndex(phys)
+
+    def _nvml_sample(self):
+        import pynvml
+        h = self.handle
+        self.rows.append((float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)),
+                          float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)),
+                          pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0,
+                          int(pynvml.nvmlDeviceGetCurrentClocksEventReasons(h))))
+
+    def _loop(self):
+        while not self.stop.wait(self.interval):
+            try:
+                self._nvml_sample()
+            except Exception:
+                return
 
     def __enter__(self):
+        try:
+            self.handle = self._nvml_handle()
+            self._nvml_sample()  # raises here, before any thread starts, when NVML cannot read the device
+            self.stop = threading.Event()
+            self.thread = threading.Thread(target=self._loop, daemon=True)
+            self.thread.start()
+            return self
+        except Exception:
+            self.thread, self.rows = None, []
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={CLOCK_FIELDS}", "--format=csv,noheader,nounits",
@@ -212,6 +263,14 @@ class ClockSampler:
         return self
 
     def __exit__(self, *exc):
+        if self.thread is not None:
+            self.stop.set()
+            self.thread.join(timeout=2)
+            try:
+                self._nvml_sample()
+            except Exception:
+                pass
+            return
         self.out = ""
         if self.proc is not None:
             time.sleep(0.2)
@@ -224,7 +283,12 @@ class ClockSampler:
 
     def summary(self):
         sm, mx, pw, reasons = [], [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for c, m, p, bits in self.rows:
+            sm.append(c)
+            mx.append(m)
+            pw.append(p)
+            reasons.update(n for n, b in self.REASON_BITS if bits & b)
+        names = [n for n, _ in self.REASON_BITS]
         for line in (self.out or "").splitlines():
             f = [x.strip() for x in line.split(",")]
             if len(f) < 9:
@@ -243,7 +307,8 @@ class ClockSampler:
         # Median over the samples taken under load (power above 30% of the highest seen).
         hot = [c for c, p in zip(sm, pw) if p >= 0.3 * max(pw)] or sm
         return {"sm_mhz": statistics.median(hot), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm), "samples_under_load": len(hot), "power_w_max": max(pw)}
+                "samples": len(sm), "samples_under_load": len(hot), "power_w_max": max(pw),
+                "source": "nvml" if self.rows else "nvidia-smi"}
 
 
 # ----------------------------------------------------------------------------- traffic record

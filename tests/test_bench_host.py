@@ -50,3 +50,18 @@ def test_replica_throughput_and_source_hash():
     assert bench.replica_throughput(5.257e12, 10, 2, 50.0) == pytest.approx(2102.8)
     h = bench._kernel_source_hash()
     assert len(h) == 16 and int(h, 16) >= 0
+
+
+def test_clock_summary_from_nvml_samples():
+    """Median SM clock over the samples under load, the maximum clock, and the
+    clock-event reasons named from NVML's bits."""
+    c = bench.ClockSampler(0)
+    c.rows = [(1965.0, 1965.0, 90.0, 0x1),          # idle sample before the region: not under load
+              (1800.0, 1965.0, 980.0, 0x4),         # sw power cap
+              (1700.0, 1965.0, 1000.0, 0x4 | 0x8),  # + hw slowdown
+              (1750.0, 1965.0, 990.0, 0x0)]
+    s = c.summary()
+    assert s["sm_mhz"] == 1750.0 and s["sm_max_mhz"] == 1965.0
+    assert s["samples"] == 4 and s["samples_under_load"] == 3
+    assert s["reasons"] == ["hw_slowdown", "sw_power_cap"] and s["source"] == "nvml"
+    assert bench.ClockSampler(0).summary()["samples"] == 0
