@@ -98,13 +98,9 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Row-major bf16 matrix [rows][cols] (cols contiguous), swizzled boxes of
-// box_cols x box_rows (128-byte swizzle unless given); out-of-range elements
-// load as zero and are not written by stores.
 // Encoded tensor maps, cached per host thread.  A map is a pure function of
-// the arguments below, so a hit returns exactly what encoding would; it saves
-// the driver call on repeated launches over the same tensors, which is most
-// of the host time of a launch-bound step.
+// the arguments below, so a hit returns exactly what encoding would, and a
+// repeated launch over the same tensors skips the driver call.
 struct TmapKey {
   const void* base;
   long long rows, cols;
@@ -130,6 +126,9 @@ int tmap_slot(const TmapKey& k) {
   return (int)((h >> 32) % kTmapCacheSlots);
 }
 
+// Row-major bf16 matrix [rows][cols] (cols contiguous), swizzled boxes of
+// box_cols x box_rows (128-byte swizzle unless given); out-of-range elements
+// load as zero and are not written by stores.
 bool make_tmap(CUtensorMap* m, const void* base, long long rows, long long cols, int box_cols, int box_rows,
                CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   const TmapKey key{base, rows, cols, box_cols, box_rows, (int)swizzle};
