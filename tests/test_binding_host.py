@@ -5,7 +5,9 @@ before anything reaches the library's compute entry points, and every entry
 point the binding names is exported by the built library.
 """
 
+import ctypes
 import os
+import re
 
 import pytest
 import torch
@@ -125,3 +127,58 @@ def test_missing_library_fails_loudly(tmp_path):
     ) % (os.path.dirname(os.path.dirname(os.path.abspath(__file__))), str(tmp_path / "absent.so"))
     out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=120).stdout
     assert out.strip() == "raised True", out
+
+
+def _header_prototypes():
+    """(return type, name, [parameter declarations]) of every function include/coda.h declares."""
+    src = open(os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "coda.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    src = "\n".join(line for line in src.splitlines() if not line.strip().startswith("#"))
+    out = []
+    for ret, name, args in re.findall(r"([A-Za-z_][\w\s*]*?)\b(coda_\w+)\s*\(([^)]*)\)\s*;", src):
+        params = [a for a in (x.strip() for x in args.split(",")) if a and a != "void"]
+        out.append((ret, name, params))
+    return out
+
+
+def _c_kind(decl: str) -> str:
+    """Kind of a C type (or of a declaration 'type name'): ptr, int, float, u64 or void."""
+    if "*" in decl:
+        return "ptr"
+    words = [w for w in decl.split() if w != "const"]
+    base = words[0] if words else ""
+    return {"int": "int", "int32_t": "int", "coda_status": "int", "float": "float", "size_t": "u64",
+            "uint64_t": "u64", "void": "void"}.get(base, base)
+
+
+def _py_kind(t) -> str:
+    if t is None:
+        return "void"
+    if t in (ctypes.c_void_p, ctypes.c_char_p) or (isinstance(t, type) and issubclass(t, ctypes._Pointer)):
+        return "ptr"
+    if t is ctypes.c_int:
+        return "int"
+    if t is ctypes.c_float:
+        return "float"
+    if t in (ctypes.c_size_t, ctypes.c_uint64):
+        return "u64"
+    return repr(t)
+
+
+def test_signatures_match_the_header():
+    """Every prototype in include/coda.h has a ctypes signature in the binding
+    with the same number and kinds of arguments and the same kind of result,
+    so the binding cannot drift from the C ABI unnoticed."""
+    protos = _header_prototypes()
+    names = {n for _, n, _ in protos}
+    assert len(protos) >= 40 and {"coda_grg_fwd", "coda_grg_bwd", "coda_swiglu_fwd", "coda_swiglu_bwd"} <= names
+    grg = next(p for _, n, p in protos if n == "coda_grg_fwd")
+    assert len(grg) == 18 and _c_kind(grg[14]) == "float"  # the parser sees eps as the 15th argument
+    lib = B.library()
+    for ret, name, params in protos:
+        fn = getattr(lib, name)
+        assert fn.argtypes is not None, f"{name}: no ctypes signature"
+        want = [_c_kind(p if p.endswith("*") else p.rsplit(" ", 1)[0]) for p in params]
+        assert [_py_kind(t) for t in fn.argtypes] == want, name
+        assert _py_kind(fn.restype) == _c_kind(ret), name
